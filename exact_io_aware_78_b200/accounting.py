@@ -1,0 +1,59 @@
+"""FLOP and byte accounting used to report throughput and roofline fractions.
+
+The forward pass does two dense contractions per attended (query, key) pair,
+S = Q K^T and O += P V, each 2*d FLOPs, so 4*d FLOPs per pair.  The
+algorithmic bytes are those of the IO-aware schedule: Q, K, V read once and
+O plus the per-row log-sum-exp written once; no N x N matrix ever moves
+(FlashAttention concept note (heepie.pages.dev), "IO complexity" table).
+"""
+from __future__ import annotations
+
+from .inputs import Workload
+
+
+def attended_pairs(N: int, causal: bool, window: int) -> int:
+    """Count pairs (i, j), 0 <= i, j < N, with (not causal or j <= i) and
+    (window <= 0 or j > i - window)."""
+    if not causal and window <= 0:
+        return N * N
+    if causal and window <= 0:
+        return N * (N + 1) // 2
+    w = min(window, N)
+    if causal:
+        # rows i < w see i + 1 keys; rows i >= w see w keys
+        return w * (w + 1) // 2 + (N - w) * w
+    # non-causal with a left bound: row i sees keys j in (i - window, N)
+    # rows i < w see all N keys; row i >= w sees N - (i - w + 1) keys
+    tail = N - w
+    return w * N + tail * N - (tail * (tail + 1)) // 2
+
+
+def flops(w: Workload) -> float:
+    """4 * d FLOPs per attended pair, summed over batch and query heads."""
+    return 4.0 * w.B * w.Hq * w.d * attended_pairs(w.N, w.causal, w.window)
+
+
+def flops_half_square(w: Workload) -> float:
+    """4*B*Hq*N^2*d, halved when causal; ignores the sliding window."""
+    f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
+    return f / 2 if w.causal else f
+
+
+def element_bytes(dtype: str) -> int:
+    return {"fp32": 4, "bf16": 2, "fp8": 1}[dtype]
+
+
+def out_bytes(dtype: str) -> int:
+    """O is fp32 for fp32 inputs and bf16 otherwise."""
+    return 4 if dtype == "fp32" else 2
+
+
+def algorithmic_bytes(w: Workload) -> int:
+    """Read Q, K, V (and fp8 scales) once; write O and the fp32 LSE once."""
+    e = element_bytes(w.dtype)
+    q = w.B * w.N * w.Hq * w.d * e
+    kv = 2 * w.B * w.N * w.Hkv * w.d * e
+    o = w.B * w.N * w.Hq * w.d * out_bytes(w.dtype)
+    lse = w.B * w.Hq * w.N * 4
+    scales = (w.Hq + 2 * w.Hkv) * 4 if w.dtype == "fp8" else 0
+    return q + kv + o + lse + scales

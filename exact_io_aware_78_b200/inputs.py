@@ -1,0 +1,133 @@
+"""Seeded synthetic inputs for the attention forward workloads.
+
+This module is shared by the CUDA path's callers (tests, bench) and by the
+float64 oracle's tests.  It holds no attention arithmetic: it draws i.i.d.
+normal tensors from a seeded CPU generator and stores them in the element
+format a workload asks for (fp32, bf16, or e4m3 codes plus per-head fp32
+scales).  Everything is generated on the CPU so that every consumer sees
+bit-identical values.
+
+Layout: Q is [B, N, Hq, d], K and V are [B, N, Hkv, d], all d-contiguous.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import torch
+
+E4M3_MAX = 448.0  # largest finite e4m3 (OCP FP8, "fn" variant) magnitude
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention-forward problem: shapes, mask, element format and seed."""
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    window: int  # <= 0: no sliding window
+    dtype: str  # "fp32" | "bf16" | "fp8"
+    seed: int
+    q_mult: float = 1.0  # Q drawn as q_mult * N(0, 1) before the format cast
+    description: str = ""
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("fp32_n128_d64", 1, 1, 1, 128, 64, False, 0, "fp32", 1234,
+                 description="non-causal, fp32 inputs, tiny"),
+        Workload("bf16_causal_b4h16_n2048_d128", 4, 16, 16, 2048, 128, True, 0, "bf16", 2048,
+                 description="causal self-attention"),
+        Workload("bf16_gqa_causal_b2h32kv8_n4096_d128_q3", 2, 32, 8, 4096, 128, True, 0, "bf16", 4096,
+                 q_mult=3.0, description="grouped-query causal, Q sharpened x3"),
+        Workload("bf16_causal_window4096_b1h16_n16384_d128", 1, 16, 16, 16384, 128, True, 4096, "bf16",
+                 16384, description="long context, causal + sliding window 4096"),
+        Workload("fp8_causal_b2h16_n8192_d128", 2, 16, 16, 8192, 128, True, 0, "fp8", 8192,
+                 description="e4m3 inputs with per-head fp32 scales"),
+    ]
+}
+
+# The workload the benchmark times by default (causal, B=4, H=16, N=2048, d=128).
+DEFAULT_BENCH_WORKLOAD = "bf16_causal_b4h16_n2048_d128"
+
+
+def _randn(seed: int, shape, mult: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    x = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if mult != 1.0:
+        x = x * mult
+    return x
+
+
+def quantize_e4m3_per_head(x: torch.Tensor):
+    """Per-head scale s_h = amax over (B, N, d) of |x[..., h, :]| / 448, codes =
+    round-to-nearest-even saturating cast of x / s_h to e4m3.  Returns
+    (codes as torch.float8_e4m3fn [same shape], scales fp32 [H])."""
+    amax = x.abs().amax(dim=(0, 1, 3)).to(torch.float32)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    codes = (x / scale.view(1, 1, -1, 1)).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return codes, scale
+
+
+def make_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, dtype: str, seed: int,
+                q_mult: float = 1.0) -> Dict[str, Optional[torch.Tensor]]:
+    """Draw Q, K, V (seeds seed, seed+1, seed+2) as fp32 N(0,1) on the CPU,
+    multiply Q by q_mult, then store them in `dtype`.
+
+    Returns a dict with CPU tensors q, k, v (dtype torch.float32,
+    torch.bfloat16 or torch.float8_e4m3fn) and q_scale, k_scale, v_scale
+    (fp32 per-head scales for fp8, else None)."""
+    q = _randn(seed + 0, (B, N, Hq, d), q_mult)
+    k = _randn(seed + 1, (B, N, Hkv, d))
+    v = _randn(seed + 2, (B, N, Hkv, d))
+    out: Dict[str, Optional[torch.Tensor]] = {"q_scale": None, "k_scale": None, "v_scale": None}
+    if dtype == "fp32":
+        out.update(q=q, k=k, v=v)
+    elif dtype == "bf16":
+        out.update(q=q.to(torch.bfloat16), k=k.to(torch.bfloat16), v=v.to(torch.bfloat16))
+    elif dtype == "fp8":
+        for name, x in (("q", q), ("k", k), ("v", v)):
+            codes, s = quantize_e4m3_per_head(x)
+            out[name] = codes
+            out[name + "_scale"] = s
+    else:
+        raise ValueError(f"unknown dtype {dtype!r}")
+    return out
+
+
+def workload_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
+    return make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.seed, w.q_mult)
+
+
+def sample_rows(N: int, window: int, count: int, seed: int):
+    """A seeded, sorted set of query rows for sampled checks at full size:
+    `count` random rows plus the first, the last, the tile edges around
+    128-row boundaries near the ends, and (with a window) the rows where the
+    window starts to bind."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    rows = set(torch.randint(0, N, (count,), generator=g).tolist())
+    rows.update({0, 1, N - 1, max(0, N - 2)})
+    for r in (127, 128, 129, 255, 256, N - 129, N - 128, N - 127):
+        if 0 <= r < N:
+            rows.add(r)
+    if window > 0:
+        for r in (window - 2, window - 1, window, window + 1):
+            if 0 <= r < N:
+                rows.add(r)
+    return sorted(rows)

@@ -1,0 +1,10 @@
+"""Float64 CPU oracle for exact attention forward (test infrastructure only).
+
+Only tests/, the package smoke check and the benchmark's CPU-baseline leg may
+import this package.  It shares no code with the CUDA path.
+"""
+from .attention import (allowed_mask, attention_ref, decode_e4m3, dequantize_per_head,
+                        online_ref, probabilities_ref)
+
+__all__ = ["allowed_mask", "attention_ref", "decode_e4m3", "dequantize_per_head",
+           "online_ref", "probabilities_ref"]

@@ -1,0 +1,79 @@
+"""Host-side checks of the seeded input recipe and the FLOP/byte accounting."""
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_78_b200 import accounting
+from exact_io_aware_78_b200.inputs import (E4M3_MAX, WORKLOADS, make_inputs,
+                                           quantize_e4m3_per_head, sample_rows)
+
+
+def test_generation_is_deterministic_and_seeded():
+    a = make_inputs(1, 2, 1, 33, 8, "bf16", 99)
+    b = make_inputs(1, 2, 1, 33, 8, "bf16", 99)
+    c = make_inputs(1, 2, 1, 33, 8, "bf16", 100)
+    for n in "qkv":
+        assert torch.equal(a[n], b[n])
+    assert not torch.equal(a["q"], c["q"])
+    assert a["q"].dtype == torch.bfloat16 and a["q"].shape == (1, 33, 2, 8)
+    assert a["k"].shape == (1, 33, 1, 8)
+
+
+def test_q_multiplier_applies_before_cast():
+    a = make_inputs(1, 1, 1, 16, 8, "fp32", 5, q_mult=3.0)
+    b = make_inputs(1, 1, 1, 16, 8, "fp32", 5)
+    assert torch.equal(a["q"], b["q"] * 3.0)
+    assert torch.equal(a["k"], b["k"])
+
+
+def test_fp8_per_head_scale_definition():
+    x = torch.randn(2, 64, 3, 16, generator=torch.Generator().manual_seed(1))
+    codes, s = quantize_e4m3_per_head(x)
+    amax = x.abs().amax(dim=(0, 1, 3))
+    torch.testing.assert_close(s, amax / E4M3_MAX)
+    deq = codes.to(torch.float32) * s.view(1, 1, -1, 1)
+    # the largest element of each head maps to +-448 exactly
+    assert torch.all(codes.to(torch.float32).abs().amax(dim=(0, 1, 3)) == E4M3_MAX)
+    # e4m3 keeps 3 mantissa bits: relative error <= 2^-4 for normal codes
+    big = x.abs() > 2 ** -6 * s.view(1, 1, -1, 1) * 4
+    rel = ((deq - x).abs() / x.abs())[big]
+    assert rel.max() <= 2 ** -4 + 1e-6
+
+
+def test_workload_table():
+    assert len(WORKLOADS) == 5
+    w = WORKLOADS["bf16_gqa_causal_b2h32kv8_n4096_d128_q3"]
+    assert (w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, w.q_mult) == (2, 32, 8, 4096, 128, True, 3.0)
+    assert w.group == 4
+
+
+@pytest.mark.parametrize("N", list(range(1, 30)) + [128, 257])
+def test_attended_pairs_brute_force(N):
+    for causal in (False, True):
+        for window in (0, 1, 2, 5, 17, 64):
+            i = np.arange(N)[:, None]
+            j = np.arange(N)[None, :]
+            ok = np.ones((N, N), bool)
+            if causal:
+                ok &= j <= i
+            if window > 0:
+                ok &= j > i - window
+            assert accounting.attended_pairs(N, causal, window) == int(ok.sum())
+
+
+def test_flop_counts_of_the_workloads():
+    w = WORKLOADS["bf16_causal_b4h16_n2048_d128"]
+    # 4*B*H*N^2*d / 2 for causal, and the exact pair count is N(N+1)/2
+    assert accounting.flops_half_square(w) == 4 * 4 * 16 * 2048 ** 2 * 128 / 2
+    assert accounting.flops(w) == 4 * 4 * 16 * 128 * (2048 * 2049 // 2)
+    w4 = WORKLOADS["bf16_causal_window4096_b1h16_n16384_d128"]
+    assert abs(accounting.flops(w4) / 1e9 - 481.05) < 0.01
+    assert abs(accounting.flops_half_square(w4) / 1e9 - 1099.51) < 0.01
+
+
+def test_sample_rows_cover_edges():
+    r = sample_rows(4096, 0, 64, 3)
+    assert r[0] == 0 and r[-1] == 4095 and 128 in r and 127 in r
+    assert r == sorted(set(r))
+    rw = sample_rows(16384, 4096, 16, 3)
+    assert 4095 in rw and 4096 in rw
