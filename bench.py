@@ -1,0 +1,390 @@
+"""Benchmark of the exact attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one attn_fwd call (every stage of the forward: tile schedule,
+TMA loads, S = Q K^T, online softmax, O += P V, epilogue) over one batch of
+the workload's seeded synthetic inputs, already resident in HBM.  Each step
+is timed with CUDA events on the launching stream; between steps a 256 MiB
+buffer is written to flush the 126 MB L2 (not timed).  Prints one JSON line.
+
+Multi-GPU (torchrun): one process per GPU, each runs its own replica of the
+workload (independent problems, no collective on the data path); the
+barrier and the max-over-ranks reduction are the only communication.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_78_b200 import accounting  # noqa: E402
+from exact_io_aware_78_b200.inputs import DEFAULT_BENCH_WORKLOAD, WORKLOADS, workload_inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh",
+                  "exact_io_aware_78_b200/csrc/exactattn.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None when there is none or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        data = json.load(f)
+    ent = data.get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.bus = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            self.bus = getattr(props, "pci_bus_id", None)
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        if not rows:
+            return None
+        bus_ids = sorted({r[0] for r in rows})
+        if self.bus is not None:
+            mine = [r for r in rows if r[0].lower().endswith(str(self.bus).lower()[-12:])]
+            rows = mine or rows
+        elif len(bus_ids) > 1:
+            # pick the busiest GPU (highest median clock) when the mapping is unknown
+            by = {b: [float(r[1]) for r in rows if r[0] == b] for b in bus_ids}
+            best = max(by, key=lambda b: statistics.median(by[b]))
+            rows = [r for r in rows if r[0] == best]
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(sm),
+                "power_w_max": max(float(r[3]) for r in rows)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------ CPU oracle arm
+def pairs_for_rows(rows, N: int, causal: bool, window: int) -> int:
+    """Attended (query, key) pairs of the given query rows."""
+    r = np.asarray(rows, dtype=np.int64)
+    hi = np.minimum(r + 1, N) if causal else np.full_like(r, N)
+    lo = np.maximum(r - window + 1, 0) if window > 0 else np.zeros_like(r)
+    return int(np.maximum(hi - lo, 0).sum())
+
+
+class OracleSampler:
+    """Times the float64 oracle on consecutive 128-row chunks of the
+    workload's (b, h) heads, continuing where the previous call stopped."""
+
+    CHUNK = 128
+
+    def __init__(self, w):
+        from oracle import dequantize_per_head  # CPU baseline leg only
+
+        self.w = w
+        inp = workload_inputs(w)
+        if w.dtype == "fp8":
+            self.qkv = [dequantize_per_head(inp[n].view(torch.uint8).numpy(), inp[n + "_scale"].numpy())
+                        for n in "qkv"]
+        else:
+            self.qkv = [inp[n].to(torch.float64).numpy() for n in "qkv"]
+        self.cursor = 0
+        self.chunks_per_head = (w.N + self.CHUNK - 1) // self.CHUNK
+
+    def run(self, budget_s: float):
+        """Returns (seconds, attended FLOPs covered, rows done)."""
+        from oracle import attention_ref  # CPU baseline leg only
+
+        w = self.w
+        g = w.Hq // w.Hkv
+        q, k, v = self.qkv
+        flops = 0.0
+        rows_done = 0
+        t0 = time.perf_counter()
+        while True:
+            idx = self.cursor % (w.B * w.Hq * self.chunks_per_head)
+            self.cursor += 1
+            bh, c = divmod(idx, self.chunks_per_head)
+            b, h = divmod(bh, w.Hq)
+            rows = list(range(c * self.CHUNK, min(w.N, (c + 1) * self.CHUNK)))
+            attention_ref(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, h // g:h // g + 1],
+                          v[b:b + 1, :, h // g:h // g + 1], w.causal, w.window, w.scale, rows=rows)
+            flops += 4.0 * w.d * pairs_for_rows(rows, w.N, w.causal, w.window)
+            rows_done += len(rows)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        return time.perf_counter() - t0, flops, rows_done
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    times = []
+    flops_done = 0.0
+    rows_total = 0
+    per_step_budget = min(20.0, 150.0 / max(1, args.steps + args.warmup))
+    sampler = OracleSampler(w)
+    for i in range(args.warmup + args.steps):
+        dt, fl, rows = sampler.run(per_step_budget)
+        if i >= args.warmup:
+            times.append(dt)
+            flops_done += fl
+            rows_total += rows
+    value = flops_done / sum(times) / 1e12
+    sample = (f"{rows_total} query rows (128-row chunks of consecutive (b,h) heads) of {w.name} over "
+              f"{args.steps} steps of ~{per_step_budget:.3g} s, numpy float64 two-pass oracle; "
+              f"TFLOP/s counts attended-pair FLOPs")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "window": w.window, "input_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- CUDA arm
+def run_cuda(args, w, world, rank, local):
+    import exact_io_aware_78_b200 as ea
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    inp = workload_inputs(w)
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    scales = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
+    o_dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
+    o = torch.empty((w.B, w.N, w.Hq, w.d), device=dev, dtype=o_dtype)
+    lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_fwd(q, k, v, o, lse, w.causal, w.window, w.scale, *scales, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st, code, site = ea.attn_get_last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {code} at site {site} during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    st, code, site = ea.attn_get_last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {code} at site {site} in the timed region")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = dist_max(sum(step_ms), world, dev)
+    flops = accounting.flops(w)
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # e2e: the public API with pinned host buffers, copies inside the timed region
+    qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    es = torch.cuda.Event(enable_timing=True)
+    ee = torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(e2e_steps + 2):
+        flush.zero_()
+        es.record(stream)
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+        ee.record(stream)
+        ee.synchronize()
+        if i >= 2:
+            e2e_ms.append(es.elapsed_time(ee))
+    e2e_total = dist_max(sum(e2e_ms), world, dev)
+    e2e_value = flops * world * e2e_steps / (e2e_total * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    bf16_peak = peaks["bf16_tflops"]
+    if w.dtype == "fp8":
+        peak = 2.0 * bf16_peak
+        peak_note = f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 dense ratio)"
+    else:
+        peak = bf16_peak
+        peak_note = f"{peak_kind} bf16 burst (kernel timed alone)"
+    launch_ms = statistics.mean(step_ms)
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    traffic = load_traffic(w.name)
+    launches_per_step = 4 if w.dtype == "fp32" else 1
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {"bf16": "bf16", "fp8": "e4m3", "fp32": "bf16x3 (fp32 in/out)"}[w.dtype],
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "window": w.window, "input_dtype": w.dtype,
+                   "flops_per_step": flops, "flops_half_square_per_step": accounting.flops_half_square(w),
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                     "algorithmic_bytes": accounting.algorithmic_bytes(w),
+                     "kernel_source_hash": kernel_source_hash()},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        dt, fl, rows = OracleSampler(w).run(args.cpu_seconds)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"{rows} query rows (128-row chunks of consecutive (b,h) heads) of "
+                                          f"{w.name} in {dt:.1f} s, numpy float64 two-pass oracle; TFLOP/s "
+                                          f"counts attended-pair FLOPs"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        # host-only: rank 0 times the oracle, other ranks exit without work
+        run_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = init_dist()
+    try:
+        run_cuda(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,624 @@
+// attn_fwd_kernel.cuh -- exact attention forward for sm_100a.
+//
+// O = softmax(scale * Q K^T + mask) V and the per-row log-sum-exp, computed
+// tile by tile in on-chip memory so that no N x N matrix reaches HBM
+// ("Flash Attention" concept note (heepie.pages.dev), "Tiling" and the TO-BE
+// diagram; FlashAttention quiz (aiunderstanding.org), questions 3-5).
+//
+// Design (B200-specific; the pages give no kernel design for this GPU):
+//   * One persistent CTA per SM walks work items (batch b, query head h,
+//     256-row query block) in a static heaviest-first order: parallelism over
+//     sequence blocks of one head ("FlashAttention-2 (PL)", "Ulepszony
+//     rownoleglosc").
+//   * A work item holds two 128-row query tiles of the same (b, h).  They
+//     share every K/V tile the TMA warp streams through a shared-memory ring,
+//     and ping-pong on the tensor core: while one tile's softmax runs on the
+//     CUDA cores, the other tile's two products run on the tensor core
+//     (asynchrony, quiz question 8 / FA-3 on the same page).
+//   * tcgen05.mma computes S = Q K^T into tensor memory (fp32); the softmax
+//     warpgroup owning the tile reads its rows (one thread per row, so row
+//     max and row sum need no cross-thread exchange: "Zoptymalizowany podzial
+//     pracy wewnatrz bloku"), applies the mask, runs exp2 with the scale
+//     folded in, keeps a running max m and sum l, writes P (bf16 or e4m3)
+//     back over S in tensor memory, and the MMA warp issues O += P V with P
+//     read straight from tensor memory.
+//   * The running max is used lazily: O and l are rescaled only when the
+//     tile max exceeds the max in use by more than kTau (log2 units), so the
+//     non-matmul work stays small ("Minimalizacja operacji nie-macierzowych").
+//   * The epilogue divides by l, converts, stores O and LSE = ln2 (m + log2 l).
+//   * Every pipeline wait is bounded: past the time limit the thread records
+//     a timeout in the device error word, raises a CTA-wide abort flag and
+//     all roles unwind; tensor memory is released and no trap is issued.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <math_constants.h>
+
+#include "sm100_ptx.cuh"
+
+namespace ea {
+
+// Device error word layout: (kind << 16) | site.
+enum : int { kErrTimeout = 1 };
+enum : int {
+  kSiteProdQEmpty = 1,
+  kSiteProdKvEmpty = 2,
+  kSiteMmaQFull = 3,
+  kSiteMmaKvFull = 4,
+  kSiteMmaPFull = 5,
+  kSiteMmaOEmpty = 6,
+  kSiteSoftSFull = 7,
+  kSiteSoftOFull = 8,
+  kSiteMmaDrain = 9,
+  kSiteProdDrain = 10
+};
+
+// Output modes of the epilogue.
+enum : int {
+  kOutBf16 = 0,      // O = acc / l (x v_scale for fp8), stored bf16
+  kOutF32Split = 1,  // O = (acc[:, :dv/2] + acc[:, dv/2:]) / l, stored fp32
+};
+
+struct FwdParams {
+  const float* q_scale;  // [Hq] (fp8 only)
+  const float* k_scale;  // [Hkv]
+  const float* v_scale;  // [Hkv]
+  void* o;               // [B, N, Hq, d_out]
+  float* lse;            // [B, Hq, N]
+  int* err;              // device error word
+  int B, Hq, Hkv, N, group;
+  int causal, window;
+  float scale_log2;      // scale * log2(e)
+  int num_qblk;          // ceil(N / 256)
+  int num_work;          // B * Hq * num_qblk
+  int order;             // 0: heaviest query blocks first, 1: lightest first
+  int skip_first_kv;     // test hook: never fill the first K/V stage
+  unsigned long long timeout_ns;
+};
+
+template <int kEsize_, int kDqk_, int kDv_, int kOut_>
+struct KernelCfg {
+  static constexpr int kEsize = kEsize_;  // bytes per input element (2 = bf16, 1 = e4m3)
+  static constexpr int kDqk = kDqk_;      // head dim of Q and K as stored
+  static constexpr int kDv = kDv_;        // head dim of V as stored (accumulator width)
+  static constexpr int kOut = kOut_;
+  static constexpr int kDout = kOut == kOutF32Split ? kDv / 2 : kDv;
+  static constexpr int BM = 128;          // query rows per tile
+  static constexpr int BN = 128;          // keys per K/V tile
+  static constexpr int kTiles = 2;        // query tiles per work item
+  // Warpgroups 0, 1: softmax of query tile 0, 1.  Warpgroup 2: warp 8 issues
+  // the MMAs, warp 9 issues the TMA copies, warps 10-11 only hold the
+  // warpgroup's register budget.  Launch budget 384 x 168 registers; the
+  // split below gives the softmax threads 224 and warpgroup 2 56:
+  // 256 * 224 + 128 * 56 = 64512 = 384 * 168.
+  static constexpr int kThreads = 384;
+  static constexpr int kSoftmaxRegs = 224;
+  static constexpr int kControlRegs = 56;
+  static constexpr int kChunkBytes = BM * 128;          // one 128-byte-wide column chunk of a tile
+  static constexpr int kChunkElems = 128 / kEsize;      // elements per 128-byte row segment
+  static constexpr int kQChunks = kDqk * kEsize / 128;
+  static constexpr int kVChunks = kDv * kEsize / 128;
+  static constexpr int kQBytes = kQChunks * kChunkBytes;
+  static constexpr int kKBytes = kQChunks * kChunkBytes;
+  static constexpr int kVBytes = kVChunks * kChunkBytes;
+  static constexpr int kStageBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
+  static constexpr int kKStep = 32 / kEsize;            // K extent of one MMA (32 bytes)
+  static constexpr int kSmemMax = 232448;               // per-CTA opt-in limit on sm_100
+  static constexpr int kBarBytes = 1024;
+  static constexpr int kStagesFit = (kSmemMax - 1024 - kBarBytes - kTiles * kQBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kQOffset = 0;
+  static constexpr int kStageOffset = kTiles * kQBytes;
+  static constexpr int kBarOffset = kStageOffset + kStages * kStageBytes;
+  static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;  // + alignment slack
+  // Tensor memory columns (fp32 accumulators; 128 lanes = 128 rows).
+  static constexpr int kTmemCols = 512;
+  __host__ __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t * 128); }
+  __host__ __device__ static constexpr uint32_t o_col(int t) { return static_cast<uint32_t>(256 + t * kDv); }
+  static constexpr float kTau = kEsize == 2 ? 8.0f : 8.0f;  // lazy-rescale threshold (log2 units)
+  static constexpr float kPShift = 0.0f;                    // P stored as 2^kPShift * p
+
+  static_assert(kDqk * kEsize % 128 == 0 && kDv * kEsize % 128 == 0, "head dims must fill 128-byte rows");
+  static_assert(kStages >= 2, "need at least two K/V stages");
+  static_assert(kDv <= 128 && kDv % 16 == 0, "accumulator width");
+  static_assert(kSmemBytes <= kSmemMax, "shared memory budget");
+  static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split over budget");
+};
+
+struct SharedCtl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t o_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SharedCtl) <= 1024, "control block");
+
+struct WorkItem {
+  int b, h, hkv, qblk;
+};
+
+struct TileRange {
+  int active;    // tile has at least one valid query row
+  int q0;        // first query row
+  int last_row;  // last valid query row
+  int lo, hi;    // K/V tile range [lo, hi) this tile visits
+};
+
+__device__ __forceinline__ WorkItem decode_work(int w, const FwdParams& p) {
+  const int bh_count = p.B * p.Hq;
+  const int r = w / bh_count;
+  const int bh = w - r * bh_count;
+  WorkItem wk;
+  wk.qblk = p.order == 0 ? (p.num_qblk - 1 - r) : r;
+  wk.b = bh / p.Hq;
+  wk.h = bh - wk.b * p.Hq;
+  wk.hkv = wk.h / p.group;
+  return wk;
+}
+
+// K/V tiles a query tile must visit: up to its last row when causal, from
+// the first key inside the first row's window when windowed.
+__device__ __forceinline__ TileRange tile_range(int qblk, int t, const FwdParams& p) {
+  TileRange r;
+  r.q0 = qblk * 256 + t * 128;
+  r.active = r.q0 < p.N;
+  r.last_row = min(r.q0 + 127, p.N - 1);
+  if (!r.active) {
+    r.lo = r.hi = 0;
+    return r;
+  }
+  const int hi_key = p.causal ? r.last_row + 1 : p.N;
+  r.hi = (hi_key + 127) / 128;
+  const int lo_key = p.window > 0 ? max(0, r.q0 - p.window + 1) : 0;
+  r.lo = lo_key / 128;
+  return r;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when the CTA is
+// aborting (another thread gave up) or when this wait ran past the time
+// limit (it then records the failure and raises the abort flag).
+__device__ __forceinline__ bool wait_phase_slow(uint32_t a, uint32_t parity, SharedCtl* ctl, const FwdParams& p,
+                                             int site, bool honor_abort) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (honor_abort && *reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+      if (globaltimer_ns() - t0 > p.timeout_ns || it > (1u << 28)) {
+        atomicCAS(p.err, 0, (kErrTimeout << 16) | site);
+        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SharedCtl* ctl, const FwdParams& p,
+                                           int site, bool honor_abort) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  return wait_phase_slow(a, parity, ctl, p, site, honor_abort);
+}
+
+// ------------------------------------------------------------- TMA producer
+template <class C>
+__device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                              const FwdParams& p, SharedCtl* ctl, uint8_t* smem) {
+  const uint64_t pol_kv = l2_policy_evict_last();
+  const uint64_t pol_q = l2_policy_evict_first();
+  uint32_t kv_pos = 0;
+  uint32_t q_iter[2] = {0, 0};
+  int skip = p.skip_first_kv;
+  uint32_t skipped_pos = 0xFFFFFFFFu;
+  bool ok = true;
+  for (int w = blockIdx.x; w < p.num_work && ok; w += gridDim.x) {
+    const WorkItem wk = decode_work(w, p);
+    TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
+    const int lo = r[0].lo;
+    const int hi = r[1].active ? r[1].hi : r[0].hi;
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!r[t].active) continue;
+      ok = wait_phase(&ctl->q_empty[t], (q_iter[t] & 1u) ^ 1u, ctl, p, kSiteProdQEmpty, true);
+      if (!ok) break;
+      ++q_iter[t];
+      mbar_arrive_expect_tx(&ctl->q_full[t], C::kQBytes);
+      uint8_t* dst = smem + C::kQOffset + t * C::kQBytes;
+#pragma unroll
+      for (int kc = 0; kc < C::kQChunks; ++kc)
+        tma_load_4d(dst + kc * C::kChunkBytes, tm_q, &ctl->q_full[t], kc * C::kChunkElems, wk.h, r[t].q0, wk.b,
+                    pol_q);
+    }
+    for (int j = lo; j < hi && ok; ++j) {
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t pos = kv_pos++;
+        const uint32_t stage = pos % C::kStages;
+        ok = wait_phase(&ctl->empty[stage], ((pos / C::kStages) & 1u) ^ 1u, ctl, p, kSiteProdKvEmpty, true);
+        if (!ok) break;
+        if (skip) {  // test hook: leave this stage unfilled
+          skip = 0;
+          skipped_pos = pos;
+          continue;
+        }
+        const int bytes = which == 0 ? C::kKBytes : C::kVBytes;
+        const int chunks = which == 0 ? C::kQChunks : C::kVChunks;
+        mbar_arrive_expect_tx(&ctl->full[stage], bytes);
+        uint8_t* dst = smem + C::kStageOffset + stage * C::kStageBytes;
+        for (int kc = 0; kc < chunks; ++kc)
+          tma_load_4d(dst + kc * C::kChunkBytes, which == 0 ? tm_k : tm_v, &ctl->full[stage],
+                      kc * C::kChunkElems, wk.hkv, j * 128, wk.b, pol_kv);
+      }
+    }
+  }
+  if (!ok) {
+    // Unwinding: wait (bounded, ignoring the abort flag) for every copy this
+    // thread started, so none lands after the CTA has exited.
+    const uint32_t first = kv_pos > C::kStages ? kv_pos - C::kStages : 0;
+    for (uint32_t pos = first; pos < kv_pos; ++pos) {
+      if (pos == skipped_pos) continue;
+      wait_phase(&ctl->full[pos % C::kStages], (pos / C::kStages) & 1u, ctl, p, kSiteProdDrain, false);
+    }
+    for (int t = 0; t < 2; ++t)
+      if (q_iter[t] > 0) wait_phase(&ctl->q_full[t], (q_iter[t] - 1) & 1u, ctl, p, kSiteProdDrain, false);
+  }
+}
+
+// ------------------------------------------------------------ MMA issuer
+template <class C>
+__device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
+  constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
+  constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
+  constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
+  const uint32_t q_addr0 = smem_u32(smem + C::kQOffset);
+  const uint32_t stage_addr0 = smem_u32(smem + C::kStageOffset);
+  uint32_t kv_pos = 0;
+  uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, o_iter[2] = {0, 0};
+  bool ok = true;
+  for (int w = blockIdx.x; w < p.num_work && ok; w += gridDim.x) {
+    const WorkItem wk = decode_work(w, p);
+    TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
+    const int lo = r[0].lo;
+    const int hi = r[1].active ? r[1].hi : r[0].hi;
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!r[t].active) continue;
+      ok = wait_phase(&ctl->q_full[t], q_phase[t], ctl, p, kSiteMmaQFull, true);
+      q_phase[t] ^= 1u;
+    }
+    if (!ok) break;
+    tc_fence_after();
+    for (int j = lo; j <= hi && ok; ++j) {
+      const uint32_t posK = kv_pos + 2u * (j - lo);  // K(j)
+      const uint32_t posV = posK - 1u;               // V(j-1)
+      if (j < hi) {
+        ok = wait_phase(&ctl->full[posK % C::kStages], (posK / C::kStages) & 1u, ctl, p, kSiteMmaKvFull, true);
+        if (!ok) break;
+      }
+      if (j > lo) {
+        ok = wait_phase(&ctl->full[posV % C::kStages], (posV / C::kStages) & 1u, ctl, p, kSiteMmaKvFull, true);
+        if (!ok) break;
+      }
+      tc_fence_after();
+      const uint32_t k_addr = stage_addr0 + (posK % C::kStages) * C::kStageBytes;
+      const uint32_t v_addr = stage_addr0 + (posV % C::kStages) * C::kStageBytes;
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const TileRange& rt = r[t];
+        if (!rt.active) continue;
+        // O_t += P_t(j-1) V(j-1)
+        if (j - 1 >= rt.lo && j - 1 < rt.hi) {
+          ok = wait_phase(&ctl->p_full[t], p_phase[t], ctl, p, kSiteMmaPFull, true);
+          p_phase[t] ^= 1u;
+          if (!ok) break;
+          if (j - 1 == rt.lo) {  // first product of this item: the previous epilogue must be done with O_t
+            ok = wait_phase(&ctl->o_empty[t], (o_iter[t] & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true);
+            ++o_iter[t];
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + C::o_col(t);
+#pragma unroll
+          for (int k = 0; k < C::BN / C::kKStep; ++k) {
+            const uint32_t a_tmem = tmem + C::s_col(t) + k * 8;
+            const uint64_t b_desc = sw128_desc(v_addr + k * C::kKStep * 128, C::kChunkBytes, 1024);
+            const uint32_t acc = (j - 1 > rt.lo || k > 0) ? 1u : 0u;
+            if (C::kEsize == 2)
+              mma_f16_ts(d_tmem, a_tmem, b_desc, kIdO, acc);
+            else
+              mma_f8_ts(d_tmem, a_tmem, b_desc, kIdO, acc);
+          }
+          if (j - 1 == rt.hi - 1) mma_commit(&ctl->o_full[t]);
+        }
+        // S_t = Q_t K(j)^T
+        if (j >= rt.lo && j < rt.hi) {
+          const uint32_t d_tmem = tmem + C::s_col(t);
+          const uint32_t qa = q_addr0 + t * C::kQBytes;
+#pragma unroll
+          for (int kc = 0; kc < C::kQChunks; ++kc) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t a_desc = sw128_desc(qa + kc * C::kChunkBytes + ks * 32, 16, 1024);
+              const uint64_t b_desc = sw128_desc(k_addr + kc * C::kChunkBytes + ks * 32, 16, 1024);
+              const uint32_t acc = (kc | ks) != 0 ? 1u : 0u;
+              if (C::kEsize == 2)
+                mma_f16_ss(d_tmem, a_desc, b_desc, kIdS, acc);
+              else
+                mma_f8_ss(d_tmem, a_desc, b_desc, kIdS, acc);
+            }
+          }
+          mma_commit(&ctl->s_full[t]);
+          if (j == rt.hi - 1) mma_commit(&ctl->q_empty[t]);
+        }
+      }
+      if (!ok) break;
+      if (j < hi) mma_commit(&ctl->empty[posK % C::kStages]);
+      if (j > lo) mma_commit(&ctl->empty[posV % C::kStages]);
+    }
+    kv_pos += 2u * (hi - lo);
+  }
+  // Every product issued so far must finish before tensor memory is freed.
+  mma_commit(&ctl->drain);
+  wait_phase(&ctl->drain, 0, ctl, p, kSiteMmaDrain, false);
+}
+
+// ------------------------------------------------------------- softmax
+template <class C>
+__device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t tmem, int warp, int lane) {
+  const int quad = warp & 3;
+  const int row_in_tile = quad * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const uint32_t tS = tmem + lane_off + C::s_col(t);
+  const uint32_t tO = tmem + lane_off + C::o_col(t);
+  uint32_t s_phase = 0, o_phase = 0;
+
+  for (int w = blockIdx.x; w < p.num_work; w += gridDim.x) {
+    const WorkItem wk = decode_work(w, p);
+    const TileRange r = tile_range(wk.qblk, t, p);
+    if (!r.active) continue;
+    const int qrow = r.q0 + row_in_tile;
+    float cs = p.scale_log2;
+    float out_mult = 1.0f;
+    if (C::kEsize == 1) {
+      cs *= __ldg(p.q_scale + wk.h) * __ldg(p.k_scale + wk.hkv);
+      out_mult = __ldg(p.v_scale + wk.hkv);
+    }
+    // Key columns this row may see: [key_lo, key_hi).
+    const int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;
+    const int key_lo = p.window > 0 ? qrow - p.window + 1 : -0x7FFFFFFF;
+
+    float m_used = -CUDART_INF_F;
+    float l = 0.0f;
+    for (int j = r.lo; j < r.hi; ++j) {
+      bool ok = wait_phase(&ctl->s_full[t], s_phase, ctl, p, kSiteSoftSFull, true);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      s_phase ^= 1u;
+      tc_fence_after();
+
+      uint32_t raw[4][32];
+      tmem_ld32(tS + 0, raw[0]);
+      tmem_ld32(tS + 32, raw[1]);
+      tmem_ld32(tS + 64, raw[2]);
+      tmem_ld32(tS + 96, raw[3]);
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
+
+      const int kbase = j * 128;
+      const bool need_mask = (kbase + 128 > p.N) || (p.causal && kbase + 127 > r.q0) ||
+                             (p.window > 0 && kbase <= r.last_row - p.window);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int col = kbase + c;
+          if (col >= key_hi || col < key_lo) s[c] = -CUDART_INF_F;
+        }
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+
+      // Lazy rescale: move the reference max only when the new tile's max
+      // exceeds it by more than kTau.
+      float alpha = 1.0f;
+      bool rescale_o = false;
+      if (m_tile > m_used + C::kTau) {
+        alpha = ex2_approx(m_used - m_tile);  // 0 when m_used is -inf
+        rescale_o = (j > r.lo) && (m_used != -CUDART_INF_F);
+        l *= alpha;
+        m_used = m_tile;
+      }
+      if (__any_sync(0xFFFFFFFFu, rescale_o)) {
+        const float f = rescale_o ? alpha : 1.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < C::kDv; cc += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + cc, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+          tmem_st32(tO + cc, ov);
+        }
+      }
+      const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used) + C::kPShift;
+
+      if (C::kEsize == 2) {
+        uint32_t pk[64];
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float p0 = ex2_approx(fmaf(s[c + 0], cs, neg_ref));
+          const float p1 = ex2_approx(fmaf(s[c + 1], cs, neg_ref));
+          const float p2 = ex2_approx(fmaf(s[c + 2], cs, neg_ref));
+          const float p3 = ex2_approx(fmaf(s[c + 3], cs, neg_ref));
+          l0 += p0;
+          l1 += p1;
+          l2 += p2;
+          l3 += p3;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+          pk[c / 2 + 1] = pack_bf16x2(p2, p3);
+        }
+        l += (l0 + l1) + (l2 + l3);
+        tmem_st32(tS + 0, &pk[0]);
+        tmem_st32(tS + 32, &pk[32]);
+      } else {
+        uint32_t pk[32];
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float p0 = ex2_approx(fmaf(s[c + 0], cs, neg_ref));
+          const float p1 = ex2_approx(fmaf(s[c + 1], cs, neg_ref));
+          const float p2 = ex2_approx(fmaf(s[c + 2], cs, neg_ref));
+          const float p3 = ex2_approx(fmaf(s[c + 3], cs, neg_ref));
+          l0 += p0;
+          l1 += p1;
+          l2 += p2;
+          l3 += p3;
+          pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
+        }
+        l += (l0 + l1) + (l2 + l3);
+        tmem_st32(tS + 0, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->p_full[t]);
+    }
+
+    // Epilogue: O = acc / l, LSE = ln 2 * (m + log2 l).
+    {
+      bool ok = wait_phase(&ctl->o_full[t], o_phase, ctl, p, kSiteSoftOFull, true);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) return;
+      o_phase ^= 1u;
+      tc_fence_after();
+      const float inv_l = l > 0.0f ? out_mult / l : 0.0f;
+      const bool store = qrow < p.N;
+      const size_t row_elem = ((static_cast<size_t>(wk.b) * p.N + qrow) * p.Hq + wk.h) * C::kDout;
+      if (C::kOut == kOutBf16) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row_elem);
+#pragma unroll 1
+        for (int cc = 0; cc < C::kDv; cc += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + cc, ov);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[cc / 8 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row_elem);
+#pragma unroll 1
+        for (int cc = 0; cc < C::kDout; cc += 32) {
+          uint32_t hi_part[32], lo_part[32];
+          tmem_ld32(tO + cc, hi_part);
+          tmem_ld32(tO + C::kDout + cc, lo_part);
+          tmem_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 v;
+              v.x = (__uint_as_float(hi_part[4 * i + 0]) + __uint_as_float(lo_part[4 * i + 0])) * inv_l;
+              v.y = (__uint_as_float(hi_part[4 * i + 1]) + __uint_as_float(lo_part[4 * i + 1])) * inv_l;
+              v.z = (__uint_as_float(hi_part[4 * i + 2]) + __uint_as_float(lo_part[4 * i + 2])) * inv_l;
+              v.w = (__uint_as_float(hi_part[4 * i + 3]) + __uint_as_float(lo_part[4 * i + 3])) * inv_l;
+              dst[cc / 4 + i] = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->o_empty[t]);
+      if (store) {
+        const float lse = l > 0.0f ? (m_used + __log2f(l) - C::kPShift) * 0.69314718055994531f
+                                   : -CUDART_INF_F;
+        p.lse[(static_cast<size_t>(wk.b) * p.Hq + wk.h) * p.N + qrow] = lse;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- the kernel
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + C::kBarOffset);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl->q_full[t], 1);
+      mbar_init(&ctl->q_empty[t], 1);
+      mbar_init(&ctl->s_full[t], 1);
+      mbar_init(&ctl->p_full[t], 4);
+      mbar_init(&ctl->o_full[t], 1);
+      mbar_init(&ctl->o_empty[t], 4);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(&ctl->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp < 8) {
+    regs_increase<C::kSoftmaxRegs>();
+    softmax_role<C>(warp >> 2, p, ctl, tmem, warp, lane);
+  } else {
+    regs_decrease<C::kControlRegs>();
+    if (warp == 8) {
+      if (lane == 0) mma_role<C>(p, ctl, smem, tmem);
+      __syncwarp();
+    } else if (warp == 9) {
+      if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, ctl, smem);
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+}  // namespace ea

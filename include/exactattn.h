@@ -1,0 +1,146 @@
+/*
+ * exactattn.h -- C ABI of the exact IO-aware attention forward for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation (Hacker News discussion item 40939398, the answer on GQA and
+ * sliding windows; "Flash Attention" concept note (heepie.pages.dev), AS-IS
+ * and TO-BE diagrams):
+ *
+ *     O   = softmax(scale * Q K^T + mask) V
+ *     LSE = per-row natural-log log-sum-exp of scale * Q K^T + mask
+ *
+ * computed tile by tile on chip with a running row maximum and row sum, so
+ * the N x N score matrix never reaches device memory (same note, "Tiling";
+ * FlashAttention quiz (aiunderstanding.org), questions 3-5).
+ *
+ * Layouts (row-major, innermost index last, no padding):
+ *     q   [B, N, Hq,  d]      k, v [B, N, Hkv, d]
+ *     o   [B, N, Hq,  d]      lse  [B, Hq, N]  (fp32)
+ * Query head h reads key/value head h / (Hq / Hkv) (grouped-query attention).
+ * Mask: key j is visible to query i iff (causal == 0 || j <= i) and
+ * (window <= 0 || j > i - window).
+ *
+ * Element formats (ea_dtype):
+ *     EA_BF16      q, k, v bf16; o bf16; fp32 accumulation.
+ *     EA_FP8_E4M3  q, k, v e4m3 codes with fp32 per-head scales q_scale[Hq],
+ *                  k_scale[Hkv], v_scale[Hkv] (real value = code * scale);
+ *                  o bf16.  The probabilities enter the second product as e4m3.
+ *     EA_FP32      q, k, v fp32; o fp32.  Each operand is split into a bf16
+ *                  high part and a bf16 remainder inside the library and the
+ *                  products hi*hi + hi*lo + lo*hi run on the bf16 tensor
+ *                  cores (d = 64 only).
+ *
+ * Ownership: every pointer passed to attn_fwd is a device pointer owned by
+ * the caller and must stay valid until the work queued on `stream` has
+ * finished.  The library owns only per-device state created on first use (an
+ * error word, cached launch attributes and, for EA_FP32, a scratch buffer for
+ * the split operands that grows to the largest size seen); attn_shutdown()
+ * frees it.
+ *
+ * Errors: functions return an ea_status.  Argument errors are detected
+ * synchronously before anything is queued.  Launches are asynchronous; a
+ * device-side failure (a pipeline wait that ran past its time limit) is
+ * recorded in the device error word and reported by attn_get_last_error().
+ * No function aborts the process or traps the GPU.
+ *
+ * Thread safety: calls for different devices may run concurrently; calls
+ * for one device are serialised by an internal lock around state creation
+ * only, and launches on one stream are ordered by that stream.
+ */
+#ifndef EXACTATTN_H
+#define EXACTATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  EA_BF16 = 0,
+  EA_FP8_E4M3 = 1,
+  EA_FP32 = 2
+} ea_dtype;
+
+typedef enum {
+  EA_OK = 0,
+  EA_EINVAL = -1,          /* bad argument: shape, null/host pointer, scale, window */
+  EA_EUNSUPPORTED = -2,    /* valid request this build has no kernel for (e.g. d = 96) */
+  EA_EALIGN = -3,          /* a pointer is not 16-byte aligned (needed by the tensor copies) */
+  EA_ELAUNCH = -4,         /* the CUDA launch itself failed */
+  EA_EDEVICE_TIMEOUT = -5, /* a device-side pipeline wait ran past its limit */
+  EA_ECUDA = -6,           /* another CUDA runtime / driver error */
+  EA_ENOMEM = -7           /* library scratch could not be allocated */
+} ea_status;
+
+/*
+ * attn_fwd -- queue one attention forward on `stream`.
+ *
+ *   q, k, v   device pointers in the layouts above, 16-byte aligned.
+ *   o         device output [B, N, Hq, d]: bf16 for EA_BF16 / EA_FP8_E4M3,
+ *             fp32 for EA_FP32.  16-byte aligned.
+ *   lse       device output [B, Hq, N] fp32 (natural log), 4-byte aligned.
+ *   B, Hq, Hkv, N, d   sizes; B, Hq, Hkv, N >= 1, Hq % Hkv == 0.
+ *             d in {64, 128} for EA_BF16 and EA_FP8_E4M3, d == 64 for EA_FP32.
+ *             Hq * N and Hkv * N must stay below 2^31.
+ *   causal    0 or 1.
+ *   window    <= 0: no sliding window; else each query sees at most the
+ *             `window` most recent keys (with causal) -- keys j > i - window.
+ *   scale     finite and > 0 (typically 1/sqrt(d)).
+ *   dtype     an ea_dtype value.
+ *   q_scale, k_scale, v_scale   device fp32 per-head scales, required for
+ *             EA_FP8_E4M3 ([Hq], [Hkv], [Hkv]); must be NULL otherwise.
+ *   stream    a cudaStream_t (NULL = legacy default stream).
+ *
+ * Returns EA_OK once the work is queued, or an error code with nothing
+ * queued.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int N, int d, int causal, int window, float scale,
+             int dtype, const float* q_scale, const float* k_scale, const float* v_scale,
+             void* stream);
+
+/*
+ * attn_get_last_error -- synchronise `stream`, then read and clear the
+ * current device's error word.  *device_code receives 0 or the recorded
+ * failure kind (1 = wait timed out), *site the pipeline wait that failed
+ * (either pointer may be NULL).  Returns EA_OK, EA_EDEVICE_TIMEOUT, or
+ * EA_ECUDA if synchronising the stream reported a CUDA error.
+ */
+int attn_get_last_error(void* stream, int* device_code, int* site);
+
+/* attn_status_string -- static, human-readable name of an ea_status. */
+const char* attn_status_string(int status);
+
+/*
+ * attn_set_option -- process-wide tuning and test hooks (host state only):
+ *   EA_OPT_WAIT_TIMEOUT_NS  limit for every device-side pipeline wait
+ *                           (default 2e9 ns).
+ *   EA_OPT_MAX_CTAS         cap on persistent CTAs per launch (0 = one per SM).
+ *   EA_OPT_SCHEDULE_ORDER   0 = heaviest query blocks first (default),
+ *                           1 = lightest first.  Results do not depend on it.
+ *   EA_OPT_SKIP_ARRIVE_ONCE test hook: the next launch's load warp skips its
+ *                           first key/value copy, so the consumer's bounded
+ *                           wait runs out and reports EA_EDEVICE_TIMEOUT.
+ * Returns EA_OK or EA_EINVAL.
+ */
+enum {
+  EA_OPT_WAIT_TIMEOUT_NS = 1,
+  EA_OPT_MAX_CTAS = 2,
+  EA_OPT_SCHEDULE_ORDER = 3,
+  EA_OPT_SKIP_ARRIVE_ONCE = 4
+};
+int attn_set_option(int option, long long value);
+
+/* attn_shutdown -- free all per-device library state (call after the
+ * streams that used it are idle).  Returns EA_OK or EA_ECUDA. */
+int attn_shutdown(void);
+
+/* attn_version -- library ABI version (major * 10000 + minor * 100 + patch). */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACTATTN_H */

@@ -1,0 +1,65 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the
+C ABI and the float64 oracle on the same seeded inputs, then compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import exact_io_aware_78_b200 as ea
+from exact_io_aware_78_b200.inputs import make_inputs
+from oracle import attention_ref, dequantize_per_head
+
+# Correctness bars: max |O - O_ref|, mean |O - O_ref|, max |LSE - LSE_ref|.
+# bf16 and fp32 inputs: 2e-2 / 2e-3 / 1e-3.  e4m3 inputs: max 6e-2; the mean
+# bar 1e-2 and LSE bar 1e-3 are derived (P enters the second product as e4m3,
+# relative step 2^-4, so per-row errors average to a few 1e-3; LSE uses fp32
+# sums of unquantised probabilities).
+TOL = {"bf16": (2e-2, 2e-3, 1e-3), "fp32": (2e-2, 2e-3, 1e-3), "fp8": (6e-2, 1e-2, 1e-3)}
+
+
+def oracle_view(inp, dtype):
+    """float64 numpy copies of exactly the values the GPU sees."""
+    if dtype == "fp8":
+        return tuple(dequantize_per_head(inp[n].view(torch.uint8).numpy(), inp[n + "_scale"].numpy())
+                     for n in "qkv")
+    return tuple(inp[n].to(torch.float64).numpy() for n in "qkv")
+
+
+def run_gpu(inp, causal, window, scale, device="cuda:0"):
+    dev = torch.device(device)
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    sc = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
+    o, lse = ea.forward(q, k, v, causal=causal, window=window, scale=scale, q_scale=sc[0], k_scale=sc[1],
+                        v_scale=sc[2])
+    st, code, site = ea.attn_get_last_error()
+    assert st == 0, f"device error code {code} at wait site {site}"
+    return o.to(torch.float64).cpu().numpy(), lse.to(torch.float64).cpu().numpy()
+
+
+def errors(O, L, Oref, Lref):
+    dO = np.abs(O - Oref)
+    dL = np.abs(L - Lref)
+    return float(dO.max()), float(dO.mean()), float(dL.max())
+
+
+def assert_close(O, L, Oref, Lref, dtype, what=""):
+    assert np.isfinite(O).all() and np.isfinite(L).all(), f"{what}: non-finite output"
+    mx, mean, lse = errors(O, L, Oref, Lref)
+    tmax, tmean, tlse = TOL[dtype]
+    msg = f"{what}: max {mx:.3e} (<= {tmax}), mean {mean:.3e} (<= {tmean}), lse {lse:.3e} (<= {tlse})"
+    print(msg)
+    assert mx <= tmax and mean <= tmean and lse <= tlse, msg
+    return mx, mean, lse
+
+
+def case(B, Hq, Hkv, N, d, causal, window, dtype, seed, q_mult=1.0, rows=None):
+    """Run one problem on the GPU and compare with the oracle (all rows, or
+    the given subset)."""
+    inp = make_inputs(B, Hq, Hkv, N, d, dtype, seed, q_mult)
+    scale = d ** -0.5
+    O, L = run_gpu(inp, causal, window, scale)
+    q, k, v = oracle_view(inp, dtype)
+    Oref, Lref = attention_ref(q, k, v, causal, window, scale, rows=rows)
+    if rows is not None:
+        O, L = O[:, rows], L[:, :, rows]
+    return assert_close(O, L, Oref, Lref, dtype, f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} c{int(causal)} w{window} {dtype}")
