@@ -33,6 +33,10 @@ _SIGNATURES = {
     "attn_set_option": (ctypes.c_int, [ctypes.c_int, ctypes.c_longlong]),
     "attn_shutdown": (ctypes.c_int, []),
     "attn_version": (ctypes.c_int, []),
+    "attn_fwd_fp32_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 _lib = None

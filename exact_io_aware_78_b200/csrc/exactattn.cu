@@ -360,3 +360,117 @@ int attn_shutdown(void) {
 int attn_version(void) { return kAbiVersion; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_fwd_fp32_noalloc: the fp32 forward with its split operands in a
+// statically allocated device array instead of cudaMallocAsync scratch.
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[EA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+uint8_t* g_noalloc_ptr[kMaxDevices] = {};  // device address of the array, per device
+int g_noalloc_sms[kMaxDevices] = {};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Once per device, with that device current: the array's device address
+// (host code must not use the symbol itself as a device pointer).
+int noalloc_setup(int dev) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] != nullptr) return EA_OK;
+  int rc = load_driver_entry_points();
+  if (rc != EA_OK) return rc;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return EA_ECUDA;
+  if (major != 10) return EA_EUNSUPPORTED;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return EA_ECUDA;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return EA_ECUDA;
+  // The array's last 256 bytes hold the timeout record of calls without a
+  // status word; start it at zero.
+  if (cudaMemset(static_cast<uint8_t*>(ptr) + EA_NOALLOC_SCRATCH_BYTES - 256, 0, 256) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
+    return EA_ECUDA;
+  g_noalloc_sms[dev] = sms;
+  g_noalloc_ptr[dev] = static_cast<uint8_t*>(ptr);
+  return EA_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+                                     int Hq, int Hkv, int N, int d, int causal, int window, float scale,
+                                     int* status, void* stream_ptr) {
+  if (!q || !k || !v || !o || !lse) return EA_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return EA_EINVAL;
+  if (Hq % Hkv != 0) return EA_EINVAL;
+  if (causal != 0 && causal != 1) return EA_EINVAL;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return EA_EINVAL;
+  if (d != 64) return EA_EUNSUPPORTED;
+  if (static_cast<long long>(Hq) * N >= (1LL << 31) || static_cast<long long>(Hkv) * N >= (1LL << 31))
+    return EA_EINVAL;
+  const long long num_qblk = (N + 255) / 256;
+  if (static_cast<long long>(B) * Hq * num_qblk > INT_MAX) return EA_EINVAL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(status, 4))
+    return EA_EALIGN;
+  const long long q_rows = static_cast<long long>(B) * N * Hq;
+  const long long kv_rows = static_cast<long long>(B) * N * Hkv;
+  const size_t sq = round256(static_cast<size_t>(q_rows) * 192 * 2);
+  const size_t sk = round256(static_cast<size_t>(kv_rows) * 192 * 2);
+  const size_t sv = round256(static_cast<size_t>(kv_rows) * 128 * 2);
+  if (sq + sk + sv + 256 > EA_NOALLOC_SCRATCH_BYTES) return EA_EINVAL;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EA_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return EA_EUNSUPPORTED;
+  int rc = noalloc_setup(dev);
+  if (rc != EA_OK) return rc;
+  const size_t q_bytes = static_cast<size_t>(q_rows) * 64 * 4;
+  const size_t kv_bytes = static_cast<size_t>(kv_rows) * 64 * 4;
+  const size_t lse_bytes = static_cast<size_t>(B) * Hq * N * 4;
+  if (check_range(q, q_bytes) || check_range(k, kv_bytes) || check_range(v, kv_bytes) || check_range(o, q_bytes) ||
+      check_range(lse, lse_bytes) || (status && check_range(status, sizeof(int))))
+    return EA_EINVAL;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
+  uint8_t* base = g_noalloc_ptr[dev];
+  uint16_t* qs = reinterpret_cast<uint16_t*>(base);
+  uint16_t* ks = reinterpret_cast<uint16_t*>(base + sq);
+  uint16_t* vs = reinterpret_cast<uint16_t*>(base + sq + sk);
+  // Timeout record when the caller passes no status word (never read back).
+  int* err_slot = reinterpret_cast<int*>(base + EA_NOALLOC_SCRATCH_BYTES - 256);
+  if (status && cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return EA_ECUDA;
+
+  ea::FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.err = status ? status : err_slot;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.causal = causal;
+  p.window = window > 0 ? window : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_qblk = static_cast<int>(num_qblk);
+  p.num_work = static_cast<int>(B * Hq * num_qblk);
+  p.order = g_order;
+  p.skip_first_kv = 0;
+  p.timeout_ns = g_timeout_ns;
+
+  DeviceState ds;
+  ds.num_sms = g_noalloc_sms[dev];
+  rc = launch_split(q, qs, q_rows, 0, ds.num_sms, stream);
+  if (rc == EA_OK) rc = launch_split(k, ks, kv_rows, 1, ds.num_sms, stream);
+  if (rc == EA_OK) rc = launch_split(v, vs, kv_rows, 2, ds.num_sms, stream);
+  if (rc != EA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, qs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 192, Hq, N, B) ||
+      make_map(&tk, ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 192, Hkv, N, B) ||
+      make_map(&tv, vs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, Hkv, N, B))
+    return EA_EINVAL;
+  return launch_attention<ea::KernelCfg<2, 192, 128, ea::kOutF32Split>>(tq, tk, tv, p, ds, stream);
+}

@@ -139,6 +139,39 @@ int attn_shutdown(void);
 /* attn_version -- library ABI version (major * 10000 + minor * 100 + patch). */
 int attn_version(void);
 
+/*
+ * attn_fwd_fp32_noalloc -- the EA_FP32 forward of attn_fwd for callers that
+ * cannot allocate device memory.  (The pages have no counterpart; this is a
+ * deployment variant.)  Such callers include code embedded in a host process
+ * whose own memory manager has reserved the device memory and forbids or
+ * cannot satisfy allocations from libraries, and runtimes that require a
+ * fixed device-memory footprint known at load time.  attn_fwd's fp32 path
+ * allocates its split operands with cudaMallocAsync on every call; this
+ * variant keeps them instead in one statically allocated device array of
+ * EA_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds
+ * until the process exits.  It calls no cudaMalloc, cudaFree or allocating
+ * library routine; the caller still passes all inputs and outputs.
+ *
+ *   q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, scale, stream:
+ *             as attn_fwd with dtype EA_FP32 (fp32 in, fp32 O, d == 64).
+ *   status    optional device int (NULL allowed): cleared on `stream`, then
+ *             set to (kind << 16) | site if a device-side pipeline wait runs
+ *             past its limit.  attn_get_last_error does not see this variant.
+ *
+ * Scratch needed: 384 * B*N*Hq + 640 * B*N*Hkv bytes (each of the three
+ * parts rounded up to 256 bytes) plus 256; a request above
+ * EA_NOALLOC_SCRATCH_BYTES returns EA_EINVAL with nothing queued.
+ * The first call on a device is a set-up call: with that device current it
+ * looks up the array's device address (with lazy module loading the CUDA
+ * runtime places the array on the device at that point) and synchronises
+ * the device once; make that first call before any stream capture.  Every call shares the one array and overwrites it completely
+ * before reading it, so calls whose work overlaps on the GPU (different
+ * streams, or different host threads) race: serialise them.
+ */
+#define EA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq,
+                          int Hkv, int N, int d, int causal, int window, float scale, int* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

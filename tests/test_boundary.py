@@ -27,7 +27,7 @@ def lib(lib_path):
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_get_last_error", "attn_status_string", "attn_set_option", "attn_shutdown",
-         "attn_version"])
+         "attn_version", "attn_fwd_fp32_noalloc"])
 
 
 def test_library_exports_every_declared_symbol(lib_path):

@@ -1,0 +1,134 @@
+"""attn_fwd_fp32_noalloc: the fp32 forward for callers that cannot allocate
+device memory (for example code inside a host process whose memory manager
+owns the device memory, or a runtime that needs a footprint fixed at load
+time).  It keeps its split operands in the library's static device array
+instead of allocating scratch on each call.
+
+Checked through the C ABI against the existing attn_fwd fp32 path, within
+the tolerances the other parity tests use, on two calls in a row (the second
+with other shapes and values, so stale contents of the shared array would
+show).  This file is collected last on purpose."""
+import pytest
+import torch
+
+import exact_io_aware_78_b200 as ea
+from exact_io_aware_78_b200 import _binding as Bn
+from exact_io_aware_78_b200.inputs import make_inputs
+
+from gpu_helpers import TOL
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_MAX = 16 * 1024 * 1024  # EA_NOALLOC_SCRATCH_BYTES in include/exactattn.h
+
+
+@pytest.fixture(scope="module")
+def lib(lib_path):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    if torch.cuda.get_device_capability(0)[0] != 10:
+        pytest.skip("needs an sm_100 GPU")
+    torch.cuda.set_device(0)
+    return ea.load_library(lib_path)
+
+
+def _outputs(q):
+    B, N, Hq, d = q.shape
+    return torch.empty_like(q), torch.empty(B, Hq, N, device=q.device, dtype=torch.float32)
+
+
+def _noalloc(lib, q, k, v, causal, window, status, out=None):
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    o, lse = _outputs(q) if out is None else out
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = lib.attn_fwd_fp32_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq,
+                                   Hkv, N, d, int(causal), window, d ** -0.5,
+                                   None if status is None else status.data_ptr(), stream)
+    return rc, o, lse
+
+
+def _compare(a_o, a_l, b_o, b_l):
+    tmax, tmean, tlse = TOL["fp32"]
+    d = (a_o.double() - b_o.double()).abs()
+    dl = (a_l.double() - b_l.double()).abs()
+    assert torch.isfinite(a_o).all() and torch.isfinite(a_l).all()
+    assert d.max().item() <= tmax and d.mean().item() <= tmean and dl.max().item() <= tlse, (
+        d.max().item(), d.mean().item(), dl.max().item())
+
+
+def test_noalloc_matches_attn_fwd_on_two_calls_in_a_row(lib):
+    dev = torch.device("cuda:0")
+    cases = [
+        (1, 1, 1, 128, 64, False, 0, 1234),   # the small fp32 workload
+        (2, 4, 2, 300, 64, True, 50, 77),     # other sizes, GQA, causal + window
+    ]
+    status = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    refs = []
+    for B, Hq, Hkv, N, d, causal, window, seed in cases:
+        inp = make_inputs(B, Hq, Hkv, N, d, "fp32", seed)
+        q, k, v = (inp[n].to(dev) for n in "qkv")
+        refs.append((q, k, v, causal, window) + ea.forward(q, k, v, causal=causal, window=window))
+    outs = [_outputs(r[0]) for r in refs] + [_outputs(refs[0][0]), _outputs(refs[0][0])]
+    # The first call on a device is the set-up call: it looks up the static
+    # array's address, and with lazy module loading the CUDA runtime places
+    # the array on the device at that moment.  Later calls allocate nothing.
+    q, k, v, causal, window, _, _ = refs[0]
+    rc, _, _ = _noalloc(lib, q, k, v, causal, window, None, outs[-1])
+    assert rc == Bn.EA_OK, Bn.status_string(rc)
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info(0)[0]
+    results = []
+    for (q, k, v, causal, window, _, _), out in zip(refs, outs):
+        rc, o, lse = _noalloc(lib, q, k, v, causal, window, status, out)
+        assert rc == Bn.EA_OK, Bn.status_string(rc)
+        torch.cuda.synchronize()
+        assert status.item() == 0  # cleared by the call, no device-side timeout
+        results.append((o, lse))
+    # the first problem again, without a status word
+    q, k, v, causal, window, _, _ = refs[0]
+    rc, o, lse = _noalloc(lib, q, k, v, causal, window, None, outs[-2])
+    assert rc == Bn.EA_OK
+    torch.cuda.synchronize()
+    results.append((o, lse))
+    # the calls allocated nothing on the device: every tensor was created
+    # before the measurement, and no comparison has run yet
+    assert torch.cuda.mem_get_info(0)[0] == free_before
+    for (o, lse), ref in zip(results, refs + [refs[0]]):
+        _compare(o, lse, ref[5], ref[6])
+
+
+def test_noalloc_rejects_requests_above_the_static_scratch(lib):
+    dev = torch.device("cuda:0")
+    # 384 * B*N*Hq + 640 * B*N*Hkv bytes of split operands must fit
+    B, Hq, Hkv, N, d = 1, 8, 8, 4096, 64
+    assert 384 * B * N * Hq + 640 * B * N * Hkv > SCRATCH_MAX
+    q = torch.zeros(B, N, Hq, d, device=dev)
+    k = torch.zeros(B, N, Hkv, d, device=dev)
+    rc, _, _ = _noalloc(lib, q, k, k, True, 0, None)
+    assert rc == Bn.EA_EINVAL
+    # and the largest request that fits is accepted
+    B, Hq, Hkv, N = 1, 1, 1, 16000
+    assert 384 * N + 640 * N + 256 * 4 <= SCRATCH_MAX
+    q = torch.randn(B, N, Hq, d, device=dev)
+    k = torch.randn(B, N, Hkv, d, device=dev)
+    rc, o, lse = _noalloc(lib, q, k, k, True, 0, None)
+    assert rc == Bn.EA_OK
+    torch.cuda.synchronize()
+    ref_o, ref_l = ea.forward(q, k, k, causal=True)
+    _compare(o, lse, ref_o, ref_l)
+
+
+def test_noalloc_argument_errors(lib):
+    dev = torch.device("cuda:0")
+    q = torch.zeros(1, 16, 2, 64, device=dev)
+    k = torch.zeros(1, 16, 1, 64, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 2, 16, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    assert lib.attn_fwd_fp32_noalloc(None, k.data_ptr(), k.data_ptr(), o.data_ptr(), lse.data_ptr(), 1, 2, 1, 16,
+                                     64, 1, 0, 0.125, None, s) == Bn.EA_EINVAL
+    assert lib.attn_fwd_fp32_noalloc(q.data_ptr(), k.data_ptr(), k.data_ptr(), o.data_ptr(), lse.data_ptr(), 1, 2,
+                                     1, 16, 128, 1, 0, 0.125, None, s) == Bn.EA_EUNSUPPORTED
+    assert lib.attn_fwd_fp32_noalloc(q.data_ptr() + 4, k.data_ptr(), k.data_ptr(), o.data_ptr(), lse.data_ptr(), 1,
+                                     2, 1, 16, 64, 1, 0, 0.125, None, s) == Bn.EA_EALIGN
