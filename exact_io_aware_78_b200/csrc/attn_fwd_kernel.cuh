@@ -90,11 +90,11 @@ struct KernelCfg {
   // Warpgroups 0, 1: softmax of query tile 0, 1.  Warpgroup 2: warp 8 issues
   // the MMAs, warp 9 issues the TMA copies, warps 10-11 only hold the
   // warpgroup's register budget.  Launch budget 384 x 168 registers; the
-  // split below gives the softmax threads 224 and warpgroup 2 56:
-  // 256 * 224 + 128 * 56 = 64512 = 384 * 168.
+  // split below gives the softmax threads 208 and warpgroup 2 88:
+  // 256 * 208 + 128 * 88 = 64512 = 384 * 168.
   static constexpr int kThreads = 384;
-  static constexpr int kSoftmaxRegs = 224;
-  static constexpr int kControlRegs = 56;
+  static constexpr int kSoftmaxRegs = 208;
+  static constexpr int kControlRegs = 88;
   static constexpr int kChunkBytes = BM * 128;          // one 128-byte-wide column chunk of a tile
   static constexpr int kChunkElems = 128 / kEsize;      // elements per 128-byte row segment
   static constexpr int kQChunks = kDqk * kEsize / 128;
@@ -150,6 +150,28 @@ struct TileRange {
   int q0;        // first query row
   int last_row;  // last valid query row
   int lo, hi;    // K/V tile range [lo, hi) this tile visits
+};
+
+// The i-th work item of this CTA.  Items are ranked heaviest first (or
+// lightest first); CTAs take them in a boustrophedon order over the ranking
+// (CTA c gets ranks c, 2G-1-c, 2G+c, 4G-1-c, ... for G CTAs), which keeps
+// the per-CTA sums of causal work within a few percent of each other.
+__device__ __forceinline__ int work_rank(int i) {
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  return i * G + ((i & 1) ? (G - 1 - c) : c);
+}
+
+// Ring position cursor over the K/V stages: stage index and mbarrier phase.
+template <int kStages>
+struct RingCursor {
+  uint32_t stage = 0, phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
 };
 
 __device__ __forceinline__ WorkItem decode_work(int w, const FwdParams& p) {
@@ -214,18 +236,24 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
                               const FwdParams& p, SharedCtl* ctl, uint8_t* smem) {
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
-  uint32_t kv_pos = 0;
+  RingCursor<C::kStages> cur;
+  uint32_t issued = 0;  // K/V positions started
   uint32_t q_iter[2] = {0, 0};
   int skip = p.skip_first_kv;
   uint32_t skipped_pos = 0xFFFFFFFFu;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.num_work && ok; w += gridDim.x) {
+  for (int i = 0; ok; ++i) {
+    const int w = work_rank(i);
+    if (w >= p.num_work) break;
     const WorkItem wk = decode_work(w, p);
-    TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
-    const int lo = r[0].lo;
-    const int hi = r[1].active ? r[1].hi : r[0].hi;
-    for (int t = 0; t < 2 && ok; ++t) {
-      if (!r[t].active) continue;
+    const TileRange r0 = tile_range(wk.qblk, 0, p);
+    const TileRange r1 = tile_range(wk.qblk, 1, p);
+    const int lo = r0.lo;
+    const int hi = r1.active ? r1.hi : r0.hi;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const TileRange& rt = t == 0 ? r0 : r1;
+      if (!ok || !rt.active) continue;
       ok = wait_phase(&ctl->q_empty[t], (q_iter[t] & 1u) ^ 1u, ctl, p, kSiteProdQEmpty, true);
       if (!ok) break;
       ++q_iter[t];
@@ -233,38 +261,44 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
       uint8_t* dst = smem + C::kQOffset + t * C::kQBytes;
 #pragma unroll
       for (int kc = 0; kc < C::kQChunks; ++kc)
-        tma_load_4d(dst + kc * C::kChunkBytes, tm_q, &ctl->q_full[t], kc * C::kChunkElems, wk.h, r[t].q0, wk.b,
+        tma_load_4d(dst + kc * C::kChunkBytes, tm_q, &ctl->q_full[t], kc * C::kChunkElems, wk.h, rt.q0, wk.b,
                     pol_q);
     }
     for (int j = lo; j < hi && ok; ++j) {
-#pragma unroll 1
+#pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t pos = kv_pos++;
-        const uint32_t stage = pos % C::kStages;
-        ok = wait_phase(&ctl->empty[stage], ((pos / C::kStages) & 1u) ^ 1u, ctl, p, kSiteProdKvEmpty, true);
         if (!ok) break;
+        ok = wait_phase(&ctl->empty[cur.stage], cur.phase ^ 1u, ctl, p, kSiteProdKvEmpty, true);
+        if (!ok) break;
+        uint64_t* full = &ctl->full[cur.stage];
+        uint8_t* dst = smem + C::kStageOffset + cur.stage * C::kStageBytes;
         if (skip) {  // test hook: leave this stage unfilled
           skip = 0;
-          skipped_pos = pos;
-          continue;
+          skipped_pos = issued;
+        } else if (which == 0) {
+          mbar_arrive_expect_tx(full, C::kKBytes);
+#pragma unroll
+          for (int kc = 0; kc < C::kQChunks; ++kc)
+            tma_load_4d(dst + kc * C::kChunkBytes, tm_k, full, kc * C::kChunkElems, wk.hkv, j * 128, wk.b, pol_kv);
+        } else {
+          mbar_arrive_expect_tx(full, C::kVBytes);
+#pragma unroll
+          for (int kc = 0; kc < C::kVChunks; ++kc)
+            tma_load_4d(dst + kc * C::kChunkBytes, tm_v, full, kc * C::kChunkElems, wk.hkv, j * 128, wk.b, pol_kv);
         }
-        const int bytes = which == 0 ? C::kKBytes : C::kVBytes;
-        const int chunks = which == 0 ? C::kQChunks : C::kVChunks;
-        mbar_arrive_expect_tx(&ctl->full[stage], bytes);
-        uint8_t* dst = smem + C::kStageOffset + stage * C::kStageBytes;
-        for (int kc = 0; kc < chunks; ++kc)
-          tma_load_4d(dst + kc * C::kChunkBytes, which == 0 ? tm_k : tm_v, &ctl->full[stage],
-                      kc * C::kChunkElems, wk.hkv, j * 128, wk.b, pol_kv);
+        ++issued;
+        cur.advance();
       }
     }
   }
   if (!ok) {
     // Unwinding: wait (bounded, ignoring the abort flag) for every copy this
-    // thread started, so none lands after the CTA has exited.
-    const uint32_t first = kv_pos > C::kStages ? kv_pos - C::kStages : 0;
-    for (uint32_t pos = first; pos < kv_pos; ++pos) {
-      if (pos == skipped_pos) continue;
-      wait_phase(&ctl->full[pos % C::kStages], (pos / C::kStages) & 1u, ctl, p, kSiteProdDrain, false);
+    // thread started, so none lands after the CTA has exited.  Only the last
+    // kStages positions can still be in flight; position P sits in stage
+    // P % kStages with phase (P / kStages) & 1.
+    for (uint32_t P = issued > C::kStages ? issued - C::kStages : 0; P < issued; ++P) {
+      if (P == skipped_pos) continue;
+      wait_phase(&ctl->full[P % C::kStages], (P / C::kStages) & 1u, ctl, p, kSiteProdDrain, false);
     }
     for (int t = 0; t < 2; ++t)
       if (q_iter[t] > 0) wait_phase(&ctl->q_full[t], (q_iter[t] - 1) & 1u, ctl, p, kSiteProdDrain, false);
@@ -272,96 +306,102 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <class C>
-__device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
+// One K/V step of query tile T: O_T += P_T(j-1) V(j-1), then S_T = Q_T K(j)^T.
+// Descriptors arrive as precomputed low halves; every MMA is one add away.
+template <class C, int T>
+__device__ __forceinline__ bool mma_tile_step(const TileRange& r, int j, uint32_t q_lo, uint32_t k_lo, uint32_t v_lo,
+                                              uint32_t tmem, SharedCtl* ctl, const FwdParams& p, uint32_t& p_phase,
+                                              uint32_t& o_iter) {
   constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
   constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
   constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
-  const uint32_t q_addr0 = smem_u32(smem + C::kQOffset);
-  const uint32_t stage_addr0 = smem_u32(smem + C::kStageOffset);
-  uint32_t kv_pos = 0;
-  uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, o_iter[2] = {0, 0};
+  constexpr uint32_t kChunkUnits = C::kChunkBytes >> 4;
+  if (r.active && j - 1 >= r.lo && j - 1 < r.hi) {
+    if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
+    p_phase ^= 1u;
+    if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
+      if (!wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
+      ++o_iter;
+    }
+    tc_fence_after();
+    const uint32_t acc0 = (j - 1 > r.lo) ? 1u : 0u;
+#pragma unroll
+    for (int k = 0; k < C::BN / C::kKStep; ++k) {
+      const uint64_t b_desc = desc_from_lo(v_lo + k * (C::kKStep * 128 / 16));
+      if (C::kEsize == 2)
+        mma_f16_ts(tmem + C::o_col(T), tmem + C::s_col(T) + k * 8, b_desc, kIdO, k == 0 ? acc0 : 1u);
+      else
+        mma_f8_ts(tmem + C::o_col(T), tmem + C::s_col(T) + k * 8, b_desc, kIdO, k == 0 ? acc0 : 1u);
+    }
+    if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
+  }
+  if (r.active && j >= r.lo && j < r.hi) {
+#pragma unroll
+    for (int kc = 0; kc < C::kQChunks; ++kc) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t a_desc = desc_from_lo(q_lo + kc * kChunkUnits + ks * 2);
+        const uint64_t b_desc = desc_from_lo(k_lo + kc * kChunkUnits + ks * 2);
+        if (C::kEsize == 2)
+          mma_f16_ss(tmem + C::s_col(T), a_desc, b_desc, kIdS, (kc | ks) != 0 ? 1u : 0u);
+        else
+          mma_f8_ss(tmem + C::s_col(T), a_desc, b_desc, kIdS, (kc | ks) != 0 ? 1u : 0u);
+      }
+    }
+    mma_commit(&ctl->s_full[T]);
+    if (j == r.hi - 1) mma_commit(&ctl->q_empty[T]);
+  }
+  return true;
+}
+
+template <class C>
+__device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
+  constexpr uint32_t kStageUnits = C::kStageBytes >> 4;
+  const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + C::kQOffset), 16);
+  const uint32_t q_lo1 = sw128_desc_lo(smem_u32(smem + C::kQOffset + C::kQBytes), 16);
+  const uint32_t k_lo_base = sw128_desc_lo(smem_u32(smem + C::kStageOffset), 16);
+  const uint32_t v_lo_base = sw128_desc_lo(smem_u32(smem + C::kStageOffset), C::kChunkBytes);
+  RingCursor<C::kStages> cur;
+  uint32_t q_phase[2] = {0, 0}, p_phase0 = 0, p_phase1 = 0, o_iter0 = 0, o_iter1 = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.num_work && ok; w += gridDim.x) {
+  for (int i = 0; ok; ++i) {
+    const int w = work_rank(i);
+    if (w >= p.num_work) break;
     const WorkItem wk = decode_work(w, p);
-    TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
-    const int lo = r[0].lo;
-    const int hi = r[1].active ? r[1].hi : r[0].hi;
-    for (int t = 0; t < 2 && ok; ++t) {
-      if (!r[t].active) continue;
-      ok = wait_phase(&ctl->q_full[t], q_phase[t], ctl, p, kSiteMmaQFull, true);
-      q_phase[t] ^= 1u;
+    const TileRange r0 = tile_range(wk.qblk, 0, p);
+    const TileRange r1 = tile_range(wk.qblk, 1, p);
+    const int lo = r0.lo;
+    const int hi = r1.active ? r1.hi : r0.hi;
+    ok = wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
+    q_phase[0] ^= 1u;
+    if (ok && r1.active) {
+      ok = wait_phase(&ctl->q_full[1], q_phase[1], ctl, p, kSiteMmaQFull, true);
+      q_phase[1] ^= 1u;
     }
     if (!ok) break;
-    tc_fence_after();
-    for (int j = lo; j <= hi && ok; ++j) {
-      const uint32_t posK = kv_pos + 2u * (j - lo);  // K(j)
-      const uint32_t posV = posK - 1u;               // V(j-1)
-      if (j < hi) {
-        ok = wait_phase(&ctl->full[posK % C::kStages], (posK / C::kStages) & 1u, ctl, p, kSiteMmaKvFull, true);
+    for (int j = lo; j <= hi; ++j) {
+      uint32_t v_stage = 0, k_stage = 0;
+      if (j > lo) {  // V(j-1) is next in ring order
+        ok = wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
+        v_stage = cur.stage;
+        cur.advance();
       }
-      if (j > lo) {
-        ok = wait_phase(&ctl->full[posV % C::kStages], (posV / C::kStages) & 1u, ctl, p, kSiteMmaKvFull, true);
+      if (j < hi) {  // then K(j)
+        ok = wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
+        k_stage = cur.stage;
+        cur.advance();
       }
       tc_fence_after();
-      const uint32_t k_addr = stage_addr0 + (posK % C::kStages) * C::kStageBytes;
-      const uint32_t v_addr = stage_addr0 + (posV % C::kStages) * C::kStageBytes;
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        const TileRange& rt = r[t];
-        if (!rt.active) continue;
-        // O_t += P_t(j-1) V(j-1)
-        if (j - 1 >= rt.lo && j - 1 < rt.hi) {
-          ok = wait_phase(&ctl->p_full[t], p_phase[t], ctl, p, kSiteMmaPFull, true);
-          p_phase[t] ^= 1u;
-          if (!ok) break;
-          if (j - 1 == rt.lo) {  // first product of this item: the previous epilogue must be done with O_t
-            ok = wait_phase(&ctl->o_empty[t], (o_iter[t] & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true);
-            ++o_iter[t];
-            if (!ok) break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + C::o_col(t);
-#pragma unroll
-          for (int k = 0; k < C::BN / C::kKStep; ++k) {
-            const uint32_t a_tmem = tmem + C::s_col(t) + k * 8;
-            const uint64_t b_desc = sw128_desc(v_addr + k * C::kKStep * 128, C::kChunkBytes, 1024);
-            const uint32_t acc = (j - 1 > rt.lo || k > 0) ? 1u : 0u;
-            if (C::kEsize == 2)
-              mma_f16_ts(d_tmem, a_tmem, b_desc, kIdO, acc);
-            else
-              mma_f8_ts(d_tmem, a_tmem, b_desc, kIdO, acc);
-          }
-          if (j - 1 == rt.hi - 1) mma_commit(&ctl->o_full[t]);
-        }
-        // S_t = Q_t K(j)^T
-        if (j >= rt.lo && j < rt.hi) {
-          const uint32_t d_tmem = tmem + C::s_col(t);
-          const uint32_t qa = q_addr0 + t * C::kQBytes;
-#pragma unroll
-          for (int kc = 0; kc < C::kQChunks; ++kc) {
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t a_desc = sw128_desc(qa + kc * C::kChunkBytes + ks * 32, 16, 1024);
-              const uint64_t b_desc = sw128_desc(k_addr + kc * C::kChunkBytes + ks * 32, 16, 1024);
-              const uint32_t acc = (kc | ks) != 0 ? 1u : 0u;
-              if (C::kEsize == 2)
-                mma_f16_ss(d_tmem, a_desc, b_desc, kIdS, acc);
-              else
-                mma_f8_ss(d_tmem, a_desc, b_desc, kIdS, acc);
-            }
-          }
-          mma_commit(&ctl->s_full[t]);
-          if (j == rt.hi - 1) mma_commit(&ctl->q_empty[t]);
-        }
-      }
+      const uint32_t k_lo = k_lo_base + k_stage * kStageUnits;
+      const uint32_t v_lo = v_lo_base + v_stage * kStageUnits;
+      ok = mma_tile_step<C, 0>(r0, j, q_lo0, k_lo, v_lo, tmem, ctl, p, p_phase0, o_iter0);
+      if (ok) ok = mma_tile_step<C, 1>(r1, j, q_lo1, k_lo, v_lo, tmem, ctl, p, p_phase1, o_iter1);
       if (!ok) break;
-      if (j < hi) mma_commit(&ctl->empty[posK % C::kStages]);
-      if (j > lo) mma_commit(&ctl->empty[posV % C::kStages]);
+      if (j < hi) mma_commit(&ctl->empty[k_stage]);
+      if (j > lo) mma_commit(&ctl->empty[v_stage]);
     }
-    kv_pos += 2u * (hi - lo);
   }
   // Every product issued so far must finish before tensor memory is freed.
   mma_commit(&ctl->drain);
@@ -378,7 +418,9 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
   const uint32_t tO = tmem + lane_off + C::o_col(t);
   uint32_t s_phase = 0, o_phase = 0;
 
-  for (int w = blockIdx.x; w < p.num_work; w += gridDim.x) {
+  for (int i = 0;; ++i) {
+    const int w = work_rank(i);
+    if (w >= p.num_work) break;
     const WorkItem wk = decode_work(w, p);
     const TileRange r = tile_range(wk.qblk, t, p);
     if (!r.active) continue;

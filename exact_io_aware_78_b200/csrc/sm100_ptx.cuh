@@ -222,6 +222,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
   return d;
 }
 
+// The same descriptor split into its 32-bit halves: the high half is the
+// same for every operand here (SBO = 1024 bytes, version 1, 128-byte
+// swizzle), and within one shared-memory tile only the start-address field
+// of the low half changes, so an operand walk is one 32-bit add.
+constexpr uint32_t kSw128DescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+  return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+
+__device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) {
+  return (static_cast<uint64_t>(kSw128DescHi) << 32) | lo;
+}
+
 // Instruction descriptor for kind::f16 / kind::f8f6f4 with fp32 accumulate.
 //   bits  4-5   D format (1 = f32)
 //   bits  7-9   A format, bits 10-12 B format
