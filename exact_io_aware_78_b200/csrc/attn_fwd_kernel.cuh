@@ -90,11 +90,11 @@ struct KernelCfg {
   // Warpgroups 0, 1: softmax of query tile 0, 1.  Warpgroup 2: warp 8 issues
   // the MMAs, warp 9 issues the TMA copies, warps 10-11 only hold the
   // warpgroup's register budget.  Launch budget 384 x 168 registers; the
-  // split below gives the softmax threads 208 and warpgroup 2 88:
-  // 256 * 208 + 128 * 88 = 64512 = 384 * 168.
+  // split below gives the softmax threads 216 and warpgroup 2 72:
+  // 256 * 216 + 128 * 72 = 64512 = 384 * 168.
   static constexpr int kThreads = 384;
-  static constexpr int kSoftmaxRegs = 208;
-  static constexpr int kControlRegs = 88;
+  static constexpr int kSoftmaxRegs = 216;
+  static constexpr int kControlRegs = 72;
   static constexpr int kChunkBytes = BM * 128;          // one 128-byte-wide column chunk of a tile
   static constexpr int kChunkElems = 128 / kEsize;      // elements per 128-byte row segment
   static constexpr int kQChunks = kDqk * kEsize / 128;
@@ -306,6 +306,34 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
 }
 
 // ------------------------------------------------------------ MMA issuer
+// O += P V over the 128 keys of a tile: BN / kKStep MMAs, A = P from tensor
+// memory (8 columns per step), B = V (MN-major, kKStep rows per step).
+template <class C, int K>
+__device__ __forceinline__ void mma_pv(uint32_t d_o, uint32_t a_p, uint32_t v_lo, uint32_t idesc, uint32_t acc0) {
+  if constexpr (K < C::BN / C::kKStep) {
+    constexpr uint32_t kOff = K * (C::kKStep * 128 / 16);
+    if constexpr (C::kEsize == 2)
+      mma_f16_ts_lo<kOff>(d_o, a_p + K * 8, v_lo, idesc, K == 0 ? acc0 : 1u);
+    else
+      mma_f8_ts_lo<kOff>(d_o, a_p + K * 8, v_lo, idesc, K == 0 ? acc0 : 1u);
+    mma_pv<C, K + 1>(d_o, a_p, v_lo, idesc, acc0);
+  }
+}
+
+// S = Q K^T over the head dimension: 4 MMAs (32 bytes of K each) per
+// 128-byte chunk, both operands K-major.
+template <class C, int I>
+__device__ __forceinline__ void mma_qk(uint32_t d_s, uint32_t q_lo, uint32_t k_lo, uint32_t idesc) {
+  if constexpr (I < C::kQChunks * 4) {
+    constexpr uint32_t kOff = (I / 4) * (C::kChunkBytes >> 4) + (I % 4) * 2;
+    if constexpr (C::kEsize == 2)
+      mma_f16_ss_lo<kOff, kOff>(d_s, q_lo, k_lo, idesc, I == 0 ? 0u : 1u);
+    else
+      mma_f8_ss_lo<kOff, kOff>(d_s, q_lo, k_lo, idesc, I == 0 ? 0u : 1u);
+    mma_qk<C, I + 1>(d_s, q_lo, k_lo, idesc);
+  }
+}
+
 // One K/V step of query tile T: O_T += P_T(j-1) V(j-1), then S_T = Q_T K(j)^T.
 // Descriptors arrive as precomputed low halves; every MMA is one add away.
 template <class C, int T>
@@ -315,7 +343,6 @@ __device__ __forceinline__ bool mma_tile_step(const TileRange& r, int j, uint32_
   constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
   constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
   constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
-  constexpr uint32_t kChunkUnits = C::kChunkBytes >> 4;
   if (r.active && j - 1 >= r.lo && j - 1 < r.hi) {
     if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
     p_phase ^= 1u;
@@ -325,29 +352,13 @@ __device__ __forceinline__ bool mma_tile_step(const TileRange& r, int j, uint32_
     }
     tc_fence_after();
     const uint32_t acc0 = (j - 1 > r.lo) ? 1u : 0u;
-#pragma unroll
-    for (int k = 0; k < C::BN / C::kKStep; ++k) {
-      const uint64_t b_desc = desc_from_lo(v_lo + k * (C::kKStep * 128 / 16));
-      if (C::kEsize == 2)
-        mma_f16_ts(tmem + C::o_col(T), tmem + C::s_col(T) + k * 8, b_desc, kIdO, k == 0 ? acc0 : 1u);
-      else
-        mma_f8_ts(tmem + C::o_col(T), tmem + C::s_col(T) + k * 8, b_desc, kIdO, k == 0 ? acc0 : 1u);
-    }
+    const uint32_t d_o = tmem + C::o_col(T);
+    const uint32_t a_p = tmem + C::s_col(T);
+    mma_pv<C, 0>(d_o, a_p, v_lo, kIdO, acc0);
     if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
   }
   if (r.active && j >= r.lo && j < r.hi) {
-#pragma unroll
-    for (int kc = 0; kc < C::kQChunks; ++kc) {
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t a_desc = desc_from_lo(q_lo + kc * kChunkUnits + ks * 2);
-        const uint64_t b_desc = desc_from_lo(k_lo + kc * kChunkUnits + ks * 2);
-        if (C::kEsize == 2)
-          mma_f16_ss(tmem + C::s_col(T), a_desc, b_desc, kIdS, (kc | ks) != 0 ? 1u : 0u);
-        else
-          mma_f8_ss(tmem + C::s_col(T), a_desc, b_desc, kIdS, (kc | ks) != 0 ? 1u : 0u);
-      }
-    }
+    mma_qk<C, 0>(tmem + C::s_col(T), q_lo, k_lo, kIdS);
     mma_commit(&ctl->s_full[T]);
     if (j == r.hi - 1) mma_commit(&ctl->q_empty[T]);
   }
@@ -409,6 +420,28 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
 }
 
 // ------------------------------------------------------------- softmax
+// Packed P words per row: bf16 pairs or e4m3 quads of 128 probabilities.
+template <class C>
+struct PWords {
+  static constexpr int kN = C::kEsize == 2 ? 64 : 32;
+};
+
+// Maximum of 128 values as a tree of three-input maxima (depth 5).
+__device__ __forceinline__ float max128(const float (&x)[128]) {
+  float a[43];
+#pragma unroll
+  for (int i = 0; i < 42; ++i) a[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+  a[42] = fmaxf(x[126], x[127]);
+  float b[15];
+#pragma unroll
+  for (int i = 0; i < 14; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[14] = a[42];
+  float c[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) c[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+  return fmaxf(fmax3(c[0], c[1], c[2]), fmaxf(c[3], c[4]));
+}
+
 template <class C>
 __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t tmem, int warp, int lane) {
   const int quad = warp & 3;
@@ -433,7 +466,7 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
     }
     // Key columns this row may see: [key_lo, key_hi).
     const int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;
-    const int key_lo = p.window > 0 ? qrow - p.window + 1 : -0x7FFFFFFF;
+    const int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
 
     float m_used = -CUDART_INF_F;
     float l = 0.0f;
@@ -444,35 +477,27 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
       s_phase ^= 1u;
       tc_fence_after();
 
-      uint32_t raw[4][32];
-      tmem_ld32(tS + 0, raw[0]);
-      tmem_ld32(tS + 32, raw[1]);
-      tmem_ld32(tS + 64, raw[2]);
-      tmem_ld32(tS + 96, raw[3]);
-      tmem_wait_ld();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
-
+      // This thread's row of S: 128 fp32 scores, one tensor-memory read.
+      float x[128];
+      {
+        uint32_t* raw = reinterpret_cast<uint32_t*>(x);
+        tmem_ld32p(tS + 0, raw);
+        tmem_ld32p(tS + 32, raw + 32);
+        tmem_ld32p(tS + 64, raw + 64);
+        tmem_ld32p(tS + 96, raw + 96);
+        tmem_wait_ld();
+      }
       const int kbase = j * 128;
       const bool need_mask = (kbase + 128 > p.N) || (p.causal && kbase + 127 > r.q0) ||
                              (p.window > 0 && kbase <= r.last_row - p.window);
       if (need_mask) {
+        const int vlo = key_lo - kbase;  // visible columns [vlo, vhi) of this tile
+        const int vhi = key_hi - kbase;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int col = kbase + c;
-          if (col >= key_hi || col < key_lo) s[c] = -CUDART_INF_F;
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c < vlo || c >= vhi) x[c] = -CUDART_INF_F;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+      const float m_tile = max128(x) * cs;
 
       // Lazy rescale: move the reference max only when the new tile's max
       // exceeds it by more than kTau.
@@ -496,44 +521,46 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
           tmem_st32(tO + cc, ov);
         }
       }
-      const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used) + C::kPShift;
 
-      if (C::kEsize == 2) {
-        uint32_t pk[64];
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // p = 2^(s cs - m): the argument in pairs, exp2 per element, the row
+      // sum in four paired partial sums, P packed and written over S.
+      {
+        const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used) + C::kPShift;
+        const uint64_t cs2 = f2_pack(cs, cs);
+        const uint64_t nr2 = f2_pack(neg_ref, neg_ref);
+        uint64_t acc[4];
+        // Two halves of 64 columns; each half's P words are stored before the
+        // next half is computed, so at most 32 packed words are live.
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float p0 = ex2_approx(fmaf(s[c + 0], cs, neg_ref));
-          const float p1 = ex2_approx(fmaf(s[c + 1], cs, neg_ref));
-          const float p2 = ex2_approx(fmaf(s[c + 2], cs, neg_ref));
-          const float p3 = ex2_approx(fmaf(s[c + 3], cs, neg_ref));
-          l0 += p0;
-          l1 += p1;
-          l2 += p2;
-          l3 += p3;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-          pk[c / 2 + 1] = pack_bf16x2(p2, p3);
-        }
-        l += (l0 + l1) + (l2 + l3);
-        tmem_st32(tS + 0, &pk[0]);
-        tmem_st32(tS + 32, &pk[32]);
-      } else {
-        uint32_t pk[32];
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[PWords<C>::kN / 2];
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float p0 = ex2_approx(fmaf(s[c + 0], cs, neg_ref));
-          const float p1 = ex2_approx(fmaf(s[c + 1], cs, neg_ref));
-          const float p2 = ex2_approx(fmaf(s[c + 2], cs, neg_ref));
-          const float p3 = ex2_approx(fmaf(s[c + 3], cs, neg_ref));
-          l0 += p0;
-          l1 += p1;
-          l2 += p2;
-          l3 += p3;
-          pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
+          for (int ii = 0; ii < 32; ++ii) {
+            const int i = h * 32 + ii;
+            const uint64_t y = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), cs2, nr2);
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            const float e0 = ex2_approx(y0);
+            const float e1 = ex2_approx(y1);
+            const uint64_t e01 = f2_pack(e0, e1);
+            acc[i & 3] = i < 4 ? e01 : f2_add(acc[i & 3], e01);
+            if (C::kEsize == 2) {
+              pk[ii] = pack_bf16x2(e0, e1);
+            } else {
+              x[2 * i] = e0;  // e4m3 packs four at a time
+              x[2 * i + 1] = e1;
+              if (ii & 1) pk[ii >> 1] = pack_e4m3x4(x[2 * i - 2], x[2 * i - 1], e0, e1);
+            }
+          }
+          if (C::kEsize == 2)
+            tmem_st32(tS + 32 * h, pk);
+          else
+            tmem_st16(tS + 16 * h, pk);
         }
-        l += (l0 + l1) + (l2 + l3);
-        tmem_st32(tS + 0, pk);
+        const uint64_t s2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float s0, s1;
+        f2_unpack(s2, s0, s1);
+        l += s0 + s1;
       }
       tmem_wait_st();
       tc_fence_before();
