@@ -23,7 +23,8 @@ constexpr int kAbiVersion = 10000;  // 1.0.0
 struct DeviceState {
   bool ready = false;
   int num_sms = 0;
-  int* err = nullptr;  // device error word
+  int* err = nullptr;             // device error word
+  cudaMemPool_t pool = nullptr;   // stream-ordered scratch for the fp32 split operands
 };
 
 std::mutex g_mutex;
@@ -72,6 +73,16 @@ int device_state(DeviceState** out) {
         return EA_ECUDA;
       if (cudaMalloc(&s.err, sizeof(int)) != cudaSuccess) return EA_ENOMEM;
       if (cudaMemset(s.err, 0, sizeof(int)) != cudaSuccess) return EA_ECUDA;
+      // A library-owned pool that keeps its memory between calls, so the
+      // per-call scratch of the fp32 path is a stream-ordered sub-allocation
+      // rather than a fresh mapping.
+      cudaMemPoolProps props{};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      if (cudaMemPoolCreate(&s.pool, &props) != cudaSuccess) return EA_ENOMEM;
+      uint64_t keep = UINT64_MAX;
+      if (cudaMemPoolSetAttribute(s.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) return EA_ECUDA;
       s.ready = true;
     }
   }
@@ -270,7 +281,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   const size_t sk = static_cast<size_t>(kv_rows) * 192 * 2;
   const size_t sv = static_cast<size_t>(kv_rows) * 128 * 2;
   void* scratch = nullptr;
-  if (cudaMallocAsync(&scratch, sq + sk + sv, stream) != cudaSuccess) return EA_ENOMEM;
+  if (cudaMallocFromPoolAsync(&scratch, sq + sk + sv, ds->pool, stream) != cudaSuccess) return EA_ENOMEM;
   uint16_t* qs = static_cast<uint16_t*>(scratch);
   uint16_t* ks = reinterpret_cast<uint16_t*>(static_cast<char*>(scratch) + sq);
   uint16_t* vs = reinterpret_cast<uint16_t*>(static_cast<char*>(scratch) + sq + sk);
@@ -350,7 +361,9 @@ int attn_shutdown(void) {
     DeviceState& s = g_dev[dev];
     if (!s.ready) continue;
     cudaSetDevice(dev);
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = EA_ECUDA;
     if (cudaFree(s.err) != cudaSuccess) rc = EA_ECUDA;
+    if (s.pool && cudaMemPoolDestroy(s.pool) != cudaSuccess) rc = EA_ECUDA;
     s = DeviceState{};
   }
   cudaSetDevice(prev);
@@ -363,7 +376,7 @@ int attn_version(void) { return kAbiVersion; }
 
 // ---------------------------------------------------------------------------
 // attn_fwd_fp32_noalloc: the fp32 forward with its split operands in a
-// statically allocated device array instead of cudaMallocAsync scratch.
+// statically allocated device array instead of pool scratch.
 namespace {
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[EA_NOALLOC_SCRATCH_BYTES];

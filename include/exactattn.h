@@ -32,10 +32,10 @@
  *
  * Ownership: every pointer passed to attn_fwd is a device pointer owned by
  * the caller and must stay valid until the work queued on `stream` has
- * finished.  The library owns only per-device state created on first use (an
- * error word, cached launch attributes and, for EA_FP32, a scratch buffer for
- * the split operands that grows to the largest size seen); attn_shutdown()
- * frees it.
+ * finished.  The library owns only per-device state created on first use: an
+ * error word, cached launch attributes, and a device memory pool from which
+ * each EA_FP32 call takes its split-operand scratch in stream order (the pool
+ * keeps its memory between calls); attn_shutdown() frees all of it.
  *
  * Errors: functions return an ea_status.  Argument errors are detected
  * synchronously before anything is queued.  Launches are asynchronous; a
@@ -146,8 +146,9 @@ int attn_version(void);
  * whose own memory manager has reserved the device memory and forbids or
  * cannot satisfy allocations from libraries, and runtimes that require a
  * fixed device-memory footprint known at load time.  attn_fwd's fp32 path
- * allocates its split operands with cudaMallocAsync on every call; this
- * variant keeps them instead in one statically allocated device array of
+ * takes its split operands from a device memory pool that the library
+ * creates and grows on demand; this variant keeps them instead in one
+ * statically allocated device array of
  * EA_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds
  * until the process exits.  It calls no cudaMalloc, cudaFree or allocating
  * library routine; the caller still passes all inputs and outputs.
