@@ -334,35 +334,35 @@ __device__ __forceinline__ void mma_qk(uint32_t d_s, uint32_t q_lo, uint32_t k_l
   }
 }
 
-// One K/V step of query tile T: O_T += P_T(j-1) V(j-1), then S_T = Q_T K(j)^T.
-// Descriptors arrive as precomputed low halves; every MMA is one add away.
+// O_T += P_T(j-1) V(j-1) for query tile T, when tile T visits K/V tile j-1.
 template <class C, int T>
-__device__ __forceinline__ bool mma_tile_step(const TileRange& r, int j, uint32_t q_lo, uint32_t k_lo, uint32_t v_lo,
-                                              uint32_t tmem, SharedCtl* ctl, const FwdParams& p, uint32_t& p_phase,
-                                              uint32_t& o_iter) {
+__device__ __forceinline__ bool mma_issue_pv(const TileRange& r, int j, uint32_t v_lo, uint32_t tmem, SharedCtl* ctl,
+                                             const FwdParams& p, uint32_t& p_phase, uint32_t& o_iter) {
   constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
-  constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
   constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
-  if (r.active && j - 1 >= r.lo && j - 1 < r.hi) {
-    if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
-    p_phase ^= 1u;
-    if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
-      if (!wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
-      ++o_iter;
-    }
-    tc_fence_after();
-    const uint32_t acc0 = (j - 1 > r.lo) ? 1u : 0u;
-    const uint32_t d_o = tmem + C::o_col(T);
-    const uint32_t a_p = tmem + C::s_col(T);
-    mma_pv<C, 0>(d_o, a_p, v_lo, kIdO, acc0);
-    if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
+  if (!(r.active && j - 1 >= r.lo && j - 1 < r.hi)) return true;
+  if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
+  p_phase ^= 1u;
+  if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
+    if (!wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
+    ++o_iter;
   }
-  if (r.active && j >= r.lo && j < r.hi) {
-    mma_qk<C, 0>(tmem + C::s_col(T), q_lo, k_lo, kIdS);
-    mma_commit(&ctl->s_full[T]);
-    if (j == r.hi - 1) mma_commit(&ctl->q_empty[T]);
-  }
+  tc_fence_after();
+  mma_pv<C, 0>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, (j - 1 > r.lo) ? 1u : 0u);
+  if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
   return true;
+}
+
+// S_T = Q_T K(j)^T for query tile T, when tile T visits K/V tile j.
+template <class C, int T>
+__device__ __forceinline__ void mma_issue_s(const TileRange& r, int j, uint32_t q_lo, uint32_t k_lo, uint32_t tmem,
+                                            SharedCtl* ctl) {
+  constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;
+  constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
+  if (!(r.active && j >= r.lo && j < r.hi)) return;
+  mma_qk<C, 0>(tmem + C::s_col(T), q_lo, k_lo, kIdS);
+  mma_commit(&ctl->s_full[T]);
+  if (j == r.hi - 1) mma_commit(&ctl->q_empty[T]);
 }
 
 template <class C>
@@ -390,6 +390,11 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
       q_phase[1] ^= 1u;
     }
     if (!ok) break;
+    // Per K/V step j: wait for V(j-1), O_0 += P_0 V(j-1), then wait for K(j)
+    // while those MMAs are still queued, S_0 = Q_0 K(j)^T, O_1 += P_1 V(j-1),
+    // release V(j-1), S_1 = Q_1 K(j)^T, release K(j).  The waits and
+    // releases sit behind queued tensor-core work, and V(j-1) goes back to
+    // the producer one batch earlier than K(j).
     for (int j = lo; j <= hi; ++j) {
       uint32_t v_stage = 0, k_stage = 0;
       if (j > lo) {  // V(j-1) is next in ring order
@@ -397,21 +402,25 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
         if (!ok) break;
         v_stage = cur.stage;
         cur.advance();
+        tc_fence_after();
       }
+      const uint32_t v_lo = v_lo_base + v_stage * kStageUnits;
+      ok = mma_issue_pv<C, 0>(r0, j, v_lo, tmem, ctl, p, p_phase0, o_iter0);
+      if (!ok) break;
       if (j < hi) {  // then K(j)
         ok = wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
         k_stage = cur.stage;
         cur.advance();
+        tc_fence_after();
       }
-      tc_fence_after();
       const uint32_t k_lo = k_lo_base + k_stage * kStageUnits;
-      const uint32_t v_lo = v_lo_base + v_stage * kStageUnits;
-      ok = mma_tile_step<C, 0>(r0, j, q_lo0, k_lo, v_lo, tmem, ctl, p, p_phase0, o_iter0);
-      if (ok) ok = mma_tile_step<C, 1>(r1, j, q_lo1, k_lo, v_lo, tmem, ctl, p, p_phase1, o_iter1);
+      mma_issue_s<C, 0>(r0, j, q_lo0, k_lo, tmem, ctl);
+      ok = mma_issue_pv<C, 1>(r1, j, v_lo, tmem, ctl, p, p_phase1, o_iter1);
       if (!ok) break;
-      if (j < hi) mma_commit(&ctl->empty[k_stage]);
       if (j > lo) mma_commit(&ctl->empty[v_stage]);
+      mma_issue_s<C, 1>(r1, j, q_lo1, k_lo, tmem, ctl);
+      if (j < hi) mma_commit(&ctl->empty[k_stage]);
     }
   }
   // Every product issued so far must finish before tensor memory is freed.
