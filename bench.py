@@ -133,11 +133,18 @@ def init_dist():
 
 
 def dist_max(x: float, world: int, device) -> float:
+    """Maximum of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tflops(flops_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own replica
+    (weak scaling), timed by the slowest rank."""
+    return flops_per_step * world * steps / (max_total_ms * 1e-3) / 1e12
 
 
 def barrier(world: int):
@@ -211,7 +218,7 @@ def run_reference(args, w, world, rank):
     times = []
     flops_done = 0.0
     rows_total = 0
-    per_step_budget = min(20.0, 150.0 / max(1, args.steps + args.warmup))
+    per_step_budget = min(20.0, args.ref_seconds / max(1, args.steps + args.warmup))
     sampler = OracleSampler(w)
     for i in range(args.warmup + args.steps):
         dt, fl, rows = sampler.run(per_step_budget)
@@ -284,7 +291,7 @@ def run_cuda(args, w, world, rank, local):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = dist_max(sum(step_ms), world, dev)
     flops = accounting.flops(w)
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(flops, args.steps, world, total_ms)
 
     # e2e: the public API with pinned host buffers, copies inside the timed region
     qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
@@ -308,7 +315,7 @@ def run_cuda(args, w, world, rank, local):
         if i >= 2:
             e2e_ms.append(es.elapsed_time(ee))
     e2e_total = dist_max(sum(e2e_ms), world, dev)
-    e2e_value = flops * world * e2e_steps / (e2e_total * 1e-3) / 1e12
+    e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
 
@@ -368,7 +375,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="host time for the cpu_baseline sample of the CUDA arm")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="total host time budget of the --impl reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
