@@ -132,6 +132,7 @@ struct SharedCtl {
   uint64_t q_full[2];
   uint64_t q_empty[2];
   uint64_t s_full[2];
+  uint64_t p_half[2];  // P of keys 0..63 stored
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t o_empty[2];
@@ -306,17 +307,18 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
 }
 
 // ------------------------------------------------------------ MMA issuer
-// O += P V over the 128 keys of a tile: BN / kKStep MMAs, A = P from tensor
-// memory (8 columns per step), B = V (MN-major, kKStep rows per step).
-template <class C, int K>
+// O += P V over keys [K0 * kKStep, K1 * kKStep) of a tile: one MMA per
+// kKStep keys, A = P from tensor memory (8 columns per step), B = V
+// (MN-major, kKStep rows per step).
+template <class C, int K, int K1>
 __device__ __forceinline__ void mma_pv(uint32_t d_o, uint32_t a_p, uint32_t v_lo, uint32_t idesc, uint32_t acc0) {
-  if constexpr (K < C::BN / C::kKStep) {
+  if constexpr (K < K1) {
     constexpr uint32_t kOff = K * (C::kKStep * 128 / 16);
     if constexpr (C::kEsize == 2)
       mma_f16_ts_lo<kOff>(d_o, a_p + K * 8, v_lo, idesc, K == 0 ? acc0 : 1u);
     else
       mma_f8_ts_lo<kOff>(d_o, a_p + K * 8, v_lo, idesc, K == 0 ? acc0 : 1u);
-    mma_pv<C, K + 1>(d_o, a_p, v_lo, idesc, acc0);
+    mma_pv<C, K + 1, K1>(d_o, a_p, v_lo, idesc, acc0);
   }
 }
 
@@ -341,14 +343,18 @@ __device__ __forceinline__ bool mma_issue_pv(const TileRange& r, int j, uint32_t
   constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
   constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
   if (!(r.active && j - 1 >= r.lo && j - 1 < r.hi)) return true;
-  if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
-  p_phase ^= 1u;
+  constexpr int kSteps = C::BN / C::kKStep;
+  if (!wait_phase(&ctl->p_half[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
   if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
     if (!wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
     ++o_iter;
   }
   tc_fence_after();
-  mma_pv<C, 0>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, (j - 1 > r.lo) ? 1u : 0u);
+  mma_pv<C, 0, kSteps / 2>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, (j - 1 > r.lo) ? 1u : 0u);
+  if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
+  p_phase ^= 1u;
+  tc_fence_after();
+  mma_pv<C, kSteps / 2, kSteps>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, 1u);
   if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
   return true;
 }
@@ -565,6 +571,12 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
             tmem_st32(tS + 32 * h, pk);
           else
             tmem_st16(tS + 16 * h, pk);
+          if (h == 0) {  // publish P of keys 0..63: the first half of P V can start
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->p_half[t]);
+          }
         }
         const uint64_t s2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         float s0, s1;
@@ -657,6 +669,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       mbar_init(&ctl->q_full[t], 1);
       mbar_init(&ctl->q_empty[t], 1);
       mbar_init(&ctl->s_full[t], 1);
+      mbar_init(&ctl->p_half[t], 4);
       mbar_init(&ctl->p_full[t], 4);
       mbar_init(&ctl->o_full[t], 1);
       mbar_init(&ctl->o_empty[t], 4);
