@@ -231,6 +231,13 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Share
   return wait_phase_slow(a, parity, ctl, p, site, honor_abort);
 }
 
+// The same for a whole warp that must stay converged (the MMA issuer): every
+// lane polls, and the warp proceeds only if every lane saw the phase.
+__device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, SharedCtl* ctl, const FwdParams& p,
+                                                int site, bool honor_abort) {
+  return __all_sync(0xFFFFFFFFu, wait_phase(bar, parity, ctl, p, site, honor_abort));
+}
+
 // ------------------------------------------------------------- TMA producer
 template <class C>
 __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
@@ -307,6 +314,9 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
 }
 
 // ------------------------------------------------------------ MMA issuer
+// One converged warp runs this role: every lane follows the same control
+// flow and waits, and elect.sync inside each MMA and commit picks lane 0
+// to issue.
 // O += P V over keys [K0 * kKStep, K1 * kKStep) of a tile: one MMA per
 // kKStep keys, A = P from tensor memory (8 columns per step), B = V
 // (MN-major, kKStep rows per step).
@@ -344,18 +354,18 @@ __device__ __forceinline__ bool mma_issue_pv(const TileRange& r, int j, uint32_t
   constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
   if (!(r.active && j - 1 >= r.lo && j - 1 < r.hi)) return true;
   constexpr int kSteps = C::BN / C::kKStep;
-  if (!wait_phase(&ctl->p_half[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
+  if (!warp_wait_phase(&ctl->p_half[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
   if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
-    if (!wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
+    if (!warp_wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
     ++o_iter;
   }
   tc_fence_after();
   mma_pv<C, 0, kSteps / 2>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, (j - 1 > r.lo) ? 1u : 0u);
-  if (!wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
+  if (!warp_wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
   p_phase ^= 1u;
   tc_fence_after();
   mma_pv<C, kSteps / 2, kSteps>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, 1u);
-  if (j - 1 == r.hi - 1) mma_commit(&ctl->o_full[T]);
+  if (j - 1 == r.hi - 1) mma_commit_elect(&ctl->o_full[T]);
   return true;
 }
 
@@ -367,8 +377,8 @@ __device__ __forceinline__ void mma_issue_s(const TileRange& r, int j, uint32_t 
   constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
   if (!(r.active && j >= r.lo && j < r.hi)) return;
   mma_qk<C, 0>(tmem + C::s_col(T), q_lo, k_lo, kIdS);
-  mma_commit(&ctl->s_full[T]);
-  if (j == r.hi - 1) mma_commit(&ctl->q_empty[T]);
+  mma_commit_elect(&ctl->s_full[T]);
+  if (j == r.hi - 1) mma_commit_elect(&ctl->q_empty[T]);
 }
 
 template <class C>
@@ -389,10 +399,10 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
     const TileRange r1 = tile_range(wk.qblk, 1, p);
     const int lo = r0.lo;
     const int hi = r1.active ? r1.hi : r0.hi;
-    ok = wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
+    ok = warp_wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
     q_phase[0] ^= 1u;
     if (ok && r1.active) {
-      ok = wait_phase(&ctl->q_full[1], q_phase[1], ctl, p, kSiteMmaQFull, true);
+      ok = warp_wait_phase(&ctl->q_full[1], q_phase[1], ctl, p, kSiteMmaQFull, true);
       q_phase[1] ^= 1u;
     }
     if (!ok) break;
@@ -404,7 +414,7 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
     for (int j = lo; j <= hi; ++j) {
       uint32_t v_stage = 0, k_stage = 0;
       if (j > lo) {  // V(j-1) is next in ring order
-        ok = wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
+        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
         v_stage = cur.stage;
         cur.advance();
@@ -414,7 +424,7 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
       ok = mma_issue_pv<C, 0>(r0, j, v_lo, tmem, ctl, p, p_phase0, o_iter0);
       if (!ok) break;
       if (j < hi) {  // then K(j)
-        ok = wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
+        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
         k_stage = cur.stage;
         cur.advance();
@@ -424,14 +434,14 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
       mma_issue_s<C, 0>(r0, j, q_lo0, k_lo, tmem, ctl);
       ok = mma_issue_pv<C, 1>(r1, j, v_lo, tmem, ctl, p, p_phase1, o_iter1);
       if (!ok) break;
-      if (j > lo) mma_commit(&ctl->empty[v_stage]);
+      if (j > lo) mma_commit_elect(&ctl->empty[v_stage]);
       mma_issue_s<C, 1>(r1, j, q_lo1, k_lo, tmem, ctl);
-      if (j < hi) mma_commit(&ctl->empty[k_stage]);
+      if (j < hi) mma_commit_elect(&ctl->empty[k_stage]);
     }
   }
   // Every product issued so far must finish before tensor memory is freed.
-  mma_commit(&ctl->drain);
-  wait_phase(&ctl->drain, 0, ctl, p, kSiteMmaDrain, false);
+  mma_commit_elect(&ctl->drain);
+  warp_wait_phase(&ctl->drain, 0, ctl, p, kSiteMmaDrain, false);
 }
 
 // ------------------------------------------------------------- softmax
@@ -698,7 +708,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   } else {
     regs_decrease<C::kControlRegs>();
     if (warp == 8) {
-      if (lane == 0) mma_role<C>(p, ctl, smem, tmem);
+      mma_role<C>(p, ctl, smem, tmem);
       __syncwarp();
     } else if (warp == 9) {
       if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, ctl, smem);
