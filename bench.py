@@ -323,11 +323,15 @@ def run_cuda(args, w, world, rank, local):
         return
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks["bf16_tflops"]
+    # The timed region runs the launches back to back; when that holds the
+    # GPU at its power cap (clocks.reasons has sw_power_cap) the sustained
+    # GEMM figure is the like-for-like denominator, so both are reported.
+    ratio = 2.0 if w.dtype == "fp8" else 1.0
+    peak = ratio * bf16_peak
+    peak_sustained = ratio * peaks["bf16_tflops_sustained"]
     if w.dtype == "fp8":
-        peak = 2.0 * bf16_peak
         peak_note = f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 dense ratio)"
     else:
-        peak = bf16_peak
         peak_note = f"{peak_kind} bf16 burst (kernel timed alone)"
     launch_ms = statistics.mean(step_ms)
     achieved = flops / (launch_ms * 1e-3) / 1e12
@@ -353,6 +357,7 @@ def run_cuda(args, w, world, rank, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                     "peak_sustained": peak_sustained, "frac_sustained": achieved / peak_sustained,
                      "algorithmic_bytes": accounting.algorithmic_bytes(w),
                      "kernel_source_hash": kernel_source_hash()},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -346,96 +346,115 @@ __device__ __forceinline__ void mma_qk(uint32_t d_s, uint32_t q_lo, uint32_t k_l
   }
 }
 
-// O_T += P_T(j-1) V(j-1) for query tile T, when tile T visits K/V tile j-1.
-template <class C, int T>
-__device__ __forceinline__ bool mma_issue_pv(const TileRange& r, int j, uint32_t v_lo, uint32_t tmem, SharedCtl* ctl,
-                                             const FwdParams& p, uint32_t& p_phase, uint32_t& o_iter) {
-  constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
-  constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
-  if (!(r.active && j - 1 >= r.lo && j - 1 < r.hi)) return true;
-  constexpr int kSteps = C::BN / C::kKStep;
-  if (!warp_wait_phase(&ctl->p_half[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
-  if (j - 1 == r.lo) {  // first product of this item: the previous epilogue must be done with O_T
-    if (!warp_wait_phase(&ctl->o_empty[T], (o_iter & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true)) return false;
-    ++o_iter;
-  }
-  tc_fence_after();
-  mma_pv<C, 0, kSteps / 2>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, (j - 1 > r.lo) ? 1u : 0u);
-  if (!warp_wait_phase(&ctl->p_full[T], p_phase, ctl, p, kSiteMmaPFull, true)) return false;
-  p_phase ^= 1u;
-  tc_fence_after();
-  mma_pv<C, kSteps / 2, kSteps>(tmem + C::o_col(T), tmem + C::s_col(T), v_lo, kIdO, 1u);
-  if (j - 1 == r.hi - 1) mma_commit_elect(&ctl->o_full[T]);
-  return true;
+// A barrier test taken ahead of time (peek) and the wait it stands for
+// (settle): the warp goes on at once when every lane's peek saw the phase
+// complete, and otherwise falls back to the bounded wait.
+__device__ __forceinline__ bool peek(uint64_t* bar, uint32_t parity) { return mbar_test_wait(smem_u32(bar), parity); }
+
+__device__ __forceinline__ bool settle(bool peeked, uint64_t* bar, uint32_t parity, SharedCtl* ctl, const FwdParams& p,
+                                       int site) {
+  if (__all_sync(0xFFFFFFFFu, peeked)) return true;
+  return warp_wait_phase(bar, parity, ctl, p, site, true);
 }
 
-// S_T = Q_T K(j)^T for query tile T, when tile T visits K/V tile j.
-template <class C, int T>
-__device__ __forceinline__ void mma_issue_s(const TileRange& r, int j, uint32_t q_lo, uint32_t k_lo, uint32_t tmem,
-                                            SharedCtl* ctl) {
-  constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;
-  constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
-  if (!(r.active && j >= r.lo && j < r.hi)) return;
-  mma_qk<C, 0>(tmem + C::s_col(T), q_lo, k_lo, kIdS);
-  mma_commit_elect(&ctl->s_full[T]);
-  if (j == r.hi - 1) mma_commit_elect(&ctl->q_empty[T]);
-}
-
+// The MMA issuer.  Per K/V step j of a work item it issues, in order:
+//   O_0 += P_0(j-1) V(j-1)  in two halves (keys 0-63 once the softmax has
+//                           published them, then keys 64-127),
+//   S_0 = Q_0 K(j)^T,
+//   O_1 += P_1(j-1) V(j-1)  in two halves,  then releases V(j-1),
+//   S_1 = Q_1 K(j)^T,                         then releases K(j).
+// S_T(j) overwrites the columns that held P_T(j-1), so it must follow
+// O_T += P_T(j-1) V(j-1) (the tensor core runs one thread's MMAs in order).
+// Every barrier the issuer needs is tested one MMA batch before it is
+// needed, so that the test's latency hides behind the MMA issue.  Waits on
+// the softmax's P and on O being free (tensor memory written or read by
+// other threads) are followed by tcgen05.fence::after_thread_sync; waits on
+// copies into shared memory need none.
 template <class C>
 __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
   constexpr uint32_t kStageUnits = C::kStageBytes >> 4;
-  const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + C::kQOffset), 16);
-  const uint32_t q_lo1 = sw128_desc_lo(smem_u32(smem + C::kQOffset + C::kQBytes), 16);
+  constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
+  constexpr uint32_t kIdO = make_idesc(kFmt, 128, C::kDv, false, true);
+  constexpr uint32_t kIdS = make_idesc(kFmt, 128, 128, false, false);
+  constexpr int kHalf = C::BN / C::kKStep / 2;  // MMAs per half of a P V product
+  const uint32_t q_lo[2] = {sw128_desc_lo(smem_u32(smem + C::kQOffset), 16),
+                            sw128_desc_lo(smem_u32(smem + C::kQOffset + C::kQBytes), 16)};
   const uint32_t k_lo_base = sw128_desc_lo(smem_u32(smem + C::kStageOffset), 16);
   const uint32_t v_lo_base = sw128_desc_lo(smem_u32(smem + C::kStageOffset), C::kChunkBytes);
   RingCursor<C::kStages> cur;
-  uint32_t q_phase[2] = {0, 0}, p_phase0 = 0, p_phase1 = 0, o_iter0 = 0, o_iter1 = 0;
+  uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, o_iter[2] = {0, 0};
   bool ok = true;
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
     const WorkItem wk = decode_work(w, p);
-    const TileRange r0 = tile_range(wk.qblk, 0, p);
-    const TileRange r1 = tile_range(wk.qblk, 1, p);
-    const int lo = r0.lo;
-    const int hi = r1.active ? r1.hi : r0.hi;
+    const TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
+    const int lo = r[0].lo;
+    const int hi = r[1].active ? r[1].hi : r[0].hi;
     ok = warp_wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
     q_phase[0] ^= 1u;
-    if (ok && r1.active) {
+    if (ok && r[1].active) {
       ok = warp_wait_phase(&ctl->q_full[1], q_phase[1], ctl, p, kSiteMmaQFull, true);
       q_phase[1] ^= 1u;
     }
     if (!ok) break;
-    // Per K/V step j: wait for V(j-1), O_0 += P_0 V(j-1), then wait for K(j)
-    // while those MMAs are still queued, S_0 = Q_0 K(j)^T, O_1 += P_1 V(j-1),
-    // release V(j-1), S_1 = Q_1 K(j)^T, release K(j).  The waits and
-    // releases sit behind queued tensor-core work, and V(j-1) goes back to
-    // the producer one batch earlier than K(j).
+    bool pk_v = false, pk_half0 = false;  // peeked during the previous step
     for (int j = lo; j <= hi; ++j) {
       uint32_t v_stage = 0, k_stage = 0;
       if (j > lo) {  // V(j-1) is next in ring order
-        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
+        ok = settle(pk_v, &ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull);
         if (!ok) break;
         v_stage = cur.stage;
         cur.advance();
-        tc_fence_after();
       }
       const uint32_t v_lo = v_lo_base + v_stage * kStageUnits;
-      ok = mma_issue_pv<C, 0>(r0, j, v_lo, tmem, ctl, p, p_phase0, o_iter0);
-      if (!ok) break;
-      if (j < hi) {  // then K(j)
-        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
-        if (!ok) break;
-        k_stage = cur.stage;
-        cur.advance();
-        tc_fence_after();
+      bool pk_k = false, pk_half1 = false;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const TileRange& rt = r[t];
+        if (rt.active && j - 1 >= rt.lo && j - 1 < rt.hi) {  // O_t += P_t(j-1) V(j-1)
+          const uint32_t d_o = tmem + C::o_col(t);
+          const uint32_t a_p = tmem + C::s_col(t);
+          ok = settle(t == 0 ? pk_half0 : pk_half1, &ctl->p_half[t], p_phase[t], ctl, p, kSiteMmaPFull);
+          if (ok && j - 1 == rt.lo) {  // first product of this item: the previous epilogue must be done with O_t
+            ok = warp_wait_phase(&ctl->o_empty[t], (o_iter[t] & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true);
+            ++o_iter[t];
+          }
+          if (!ok) break;
+          tc_fence_after();
+          const bool pk_full = peek(&ctl->p_full[t], p_phase[t]);
+          mma_pv<C, 0, kHalf>(d_o, a_p, v_lo, kIdO, (j - 1 > rt.lo) ? 1u : 0u);
+          ok = settle(pk_full, &ctl->p_full[t], p_phase[t], ctl, p, kSiteMmaPFull);
+          if (!ok) break;
+          p_phase[t] ^= 1u;
+          tc_fence_after();
+          if (t == 0 && j < hi) pk_k = peek(&ctl->full[cur.stage], cur.phase);
+          mma_pv<C, kHalf, 2 * kHalf>(d_o, a_p, v_lo, kIdO, 1u);
+          if (j - 1 == rt.hi - 1) mma_commit_elect(&ctl->o_full[t]);
+        }
+        if (t == 0) {
+          if (j < hi) {  // K(j)
+            ok = settle(pk_k, &ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull);
+            if (!ok) break;
+            k_stage = cur.stage;
+            cur.advance();
+          }
+          if (r[1].active && j - 1 >= r[1].lo && j - 1 < r[1].hi) pk_half1 = peek(&ctl->p_half[1], p_phase[1]);
+        } else if (j > lo) {
+          mma_commit_elect(&ctl->empty[v_stage]);
+          // for the next step: V(j), next in ring order, and P_0(j)
+          if (j < hi) {
+            pk_v = peek(&ctl->full[cur.stage], cur.phase);
+            if (r[0].active && j >= r[0].lo && j < r[0].hi) pk_half0 = peek(&ctl->p_half[0], p_phase[0]);
+          }
+        }
+        if (rt.active && j >= rt.lo && j < rt.hi) {  // S_t = Q_t K(j)^T
+          mma_qk<C, 0>(tmem + C::s_col(t), q_lo[t], k_lo_base + k_stage * kStageUnits, kIdS);
+          mma_commit_elect(&ctl->s_full[t]);
+          if (j == rt.hi - 1) mma_commit_elect(&ctl->q_empty[t]);
+        }
       }
-      const uint32_t k_lo = k_lo_base + k_stage * kStageUnits;
-      mma_issue_s<C, 0>(r0, j, q_lo0, k_lo, tmem, ctl);
-      ok = mma_issue_pv<C, 1>(r1, j, v_lo, tmem, ctl, p, p_phase1, o_iter1);
       if (!ok) break;
-      if (j > lo) mma_commit_elect(&ctl->empty[v_stage]);
-      mma_issue_s<C, 1>(r1, j, q_lo1, k_lo, tmem, ctl);
       if (j < hi) mma_commit_elect(&ctl->empty[k_stage]);
     }
   }
