@@ -93,6 +93,7 @@ struct KernelCfg {
   // split below gives the softmax threads 216 and warpgroup 2 72:
   // 256 * 216 + 128 * 72 = 64512 = 384 * 168.
   static constexpr int kThreads = 384;
+  static constexpr int kLaunchRegs = 168;
   static constexpr int kSoftmaxRegs = 216;
   static constexpr int kControlRegs = 72;
   static constexpr int kChunkBytes = BM * 128;          // one 128-byte-wide column chunk of a tile
@@ -123,7 +124,8 @@ struct KernelCfg {
   static_assert(kStages >= 2, "need at least two K/V stages");
   static_assert(kDv <= 128 && kDv % 16 == 0, "accumulator width");
   static_assert(kSmemBytes <= kSmemMax, "shared memory budget");
-  static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split over budget");
+  static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split over budget");
+  static_assert(kLaunchRegs * kThreads <= 65536, "launch register budget");
 };
 
 struct SharedCtl {

@@ -128,6 +128,12 @@ int launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     if (cudaFuncSetAttribute(ea::attn_fwd_sm100<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
       return EA_ELAUNCH;
+    // The warpgroups re-split the registers the block is launched with
+    // (setmaxnreg); a block launched with fewer than the split assumes would
+    // wait in setmaxnreg forever, so refuse to launch it.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, ea::attn_fwd_sm100<C>) != cudaSuccess || fa.numRegs < C::kLaunchRegs)
+      return EA_ELAUNCH;
     attr_done[dev] = true;
   }
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
@@ -140,22 +146,33 @@ int launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 // kernel then sees Q' = [hi, hi, lo], K' = [hi, lo, hi] (so that
 // Q' K'^T = Qh Kh^T + Qh Kl^T + Ql Kh^T) and V' = [hi, lo] (so that
 // P V' = [P Vh, P Vl], summed in the epilogue).
-__global__ void split_fp32_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, long long rows,
-                                  int pattern /*0: Q, 1: K, 2: V*/) {
-  // One thread per group of 8 consecutive elements of a 64-wide row.
-  const long long groups = rows * 8;
+struct SplitJob {
+  const float* x;
+  uint16_t* y;
+  long long rows;
+};
+
+// One launch splits Q, K and V: a grid-stride loop over groups of 8
+// consecutive elements of 64-wide rows, Q's groups first, then K's, then V's.
+__global__ void split_fp32_kernel(SplitJob q, SplitJob k, SplitJob v) {
+  const long long gq = q.rows * 8, gk = k.rows * 8;
+  const long long groups = gq + gk + v.rows * 8;
   for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
        g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = g >> 3;
-    const int col = static_cast<int>(g & 7) * 8;
+    const int pattern = g < gq ? 0 : (g < gq + gk ? 1 : 2);  // 0: Q, 1: K, 2: V
+    const float* x = pattern == 0 ? q.x : (pattern == 1 ? k.x : v.x);
+    uint16_t* y = pattern == 0 ? q.y : (pattern == 1 ? k.y : v.y);
+    const long long gl = g - (pattern == 0 ? 0 : (pattern == 1 ? gq : gq + gk));
+    const long long row = gl >> 3;
+    const int col = static_cast<int>(gl & 7) * 8;
     const float4* src = reinterpret_cast<const float4*>(x + row * 64 + col);
     const float4 a = src[0], b = src[1];
-    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const float vals[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     uint16_t hi[8], lo[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
-      const __nv_bfloat16 l = __float2bfloat16_rn(v[i] - __bfloat162float(h));
+      const __nv_bfloat16 h = __float2bfloat16_rn(vals[i]);
+      const __nv_bfloat16 l = __float2bfloat16_rn(vals[i] - __bfloat162float(h));
       hi[i] = *reinterpret_cast<const uint16_t*>(&h);
       lo[i] = *reinterpret_cast<const uint16_t*>(&l);
     }
@@ -176,12 +193,12 @@ __global__ void split_fp32_kernel(const float* __restrict__ x, uint16_t* __restr
   }
 }
 
-int launch_split(const float* x, uint16_t* y, long long rows, int pattern, int num_sms, cudaStream_t stream) {
-  const long long groups = rows * 8;
+int launch_split(SplitJob q, SplitJob k, SplitJob v, int num_sms, cudaStream_t stream) {
+  const long long groups = (q.rows + k.rows + v.rows) * 8;
   long long blocks = (groups + 255) / 256;
   if (blocks > 8LL * num_sms) blocks = 8LL * num_sms;
   if (blocks < 1) blocks = 1;
-  split_fp32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, y, rows, pattern);
+  split_fp32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(q, k, v);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
 }
 
@@ -285,9 +302,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   uint16_t* qs = static_cast<uint16_t*>(scratch);
   uint16_t* ks = reinterpret_cast<uint16_t*>(static_cast<char*>(scratch) + sq);
   uint16_t* vs = reinterpret_cast<uint16_t*>(static_cast<char*>(scratch) + sq + sk);
-  rc = launch_split(static_cast<const float*>(q), qs, q_rows, 0, ds->num_sms, stream);
-  if (rc == EA_OK) rc = launch_split(static_cast<const float*>(k), ks, kv_rows, 1, ds->num_sms, stream);
-  if (rc == EA_OK) rc = launch_split(static_cast<const float*>(v), vs, kv_rows, 2, ds->num_sms, stream);
+  rc = launch_split({static_cast<const float*>(q), qs, q_rows}, {static_cast<const float*>(k), ks, kv_rows},
+                    {static_cast<const float*>(v), vs, kv_rows}, ds->num_sms, stream);
   if (rc == EA_OK) {
     if (make_map(&tq, qs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 192, Hq, N, B) ||
         make_map(&tk, ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 192, Hkv, N, B) ||
@@ -476,9 +492,7 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
 
   DeviceState ds;
   ds.num_sms = g_noalloc_sms[dev];
-  rc = launch_split(q, qs, q_rows, 0, ds.num_sms, stream);
-  if (rc == EA_OK) rc = launch_split(k, ks, kv_rows, 1, ds.num_sms, stream);
-  if (rc == EA_OK) rc = launch_split(v, vs, kv_rows, 2, ds.num_sms, stream);
+  rc = launch_split({q, qs, q_rows}, {k, ks, kv_rows}, {v, vs, kv_rows}, ds.num_sms, stream);
   if (rc != EA_OK) return rc;
   CUtensorMap tq, tk, tv;
   if (make_map(&tq, qs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 192, Hq, N, B) ||
