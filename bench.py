@@ -30,7 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_78_b200 import accounting  # noqa: E402
-from exact_io_aware_78_b200.inputs import DEFAULT_BENCH_WORKLOAD, WORKLOADS, workload_inputs  # noqa: E402
+from exact_io_aware_78_b200.inputs import (DEFAULT_BENCH_WORKLOAD, WORKLOADS, head_shard,  # noqa: E402
+                                           shard_inputs, workload_inputs)
 
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -147,6 +148,12 @@ def job_tflops(flops_per_step: float, steps: int, world: int, max_total_ms: floa
     return flops_per_step * world * steps / (max_total_ms * 1e-3) / 1e12
 
 
+def sharded_tflops(job_flops_per_step: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput when the ranks split one problem's heads (strong
+    scaling): the full problem's FLOPs per step over the slowest rank's time."""
+    return job_flops_per_step * steps / (max_total_ms * 1e-3) / 1e12
+
+
 def barrier(world: int):
     if world > 1:
         torch.distributed.barrier()
@@ -250,7 +257,11 @@ def run_cuda(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     ea.load_library()
+    w_job = w
     inp = workload_inputs(w)
+    if args.shard == "heads":
+        w, q_lo, q_hi, kv_lo, kv_hi = head_shard(w_job, world, rank)
+        inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
     q, k, v = (inp[n].to(dev) for n in "qkv")
     scales = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
     o_dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
@@ -290,8 +301,11 @@ def run_cuda(args, w, world, rank, local):
         raise RuntimeError(f"device error {code} at site {site} in the timed region")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = dist_max(sum(step_ms), world, dev)
-    flops = accounting.flops(w)
-    value = job_tflops(flops, args.steps, world, total_ms)
+    flops = accounting.flops(w)  # this rank's launch
+    if args.shard == "heads":
+        value = sharded_tflops(accounting.flops(w_job), args.steps, total_ms)
+    else:
+        value = job_tflops(flops, args.steps, world, total_ms)
 
     # e2e: the public API with pinned host buffers, copies inside the timed region
     qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
@@ -315,7 +329,10 @@ def run_cuda(args, w, world, rank, local):
         if i >= 2:
             e2e_ms.append(es.elapsed_time(ee))
     e2e_total = dist_max(sum(e2e_ms), world, dev)
-    e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
+    if args.shard == "heads":
+        e2e_value = sharded_tflops(accounting.flops(w_job), e2e_steps, e2e_total)
+    else:
+        e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
 
@@ -346,15 +363,18 @@ def run_cuda(args, w, world, rank, local):
         "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "fp8": "e4m3", "fp32": "bf16x3 (fp32 in/out)"}[w.dtype],
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-                   "causal": w.causal, "window": w.window, "input_dtype": w.dtype,
-                   "flops_per_step": flops, "flops_half_square_per_step": accounting.flops_half_square(w),
+        "config": {"workload": w_job.name, "B": w_job.B, "Hq": w_job.Hq, "Hkv": w_job.Hkv, "N": w_job.N,
+                   "d": w_job.d, "causal": w_job.causal, "window": w_job.window, "input_dtype": w_job.dtype,
+                   "flops_per_step": accounting.flops(w_job),
+                   "flops_half_square_per_step": accounting.flops_half_square(w_job),
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": (f"head shards x{world} (rank 0: query heads {w.Hq}, kv heads {w.Hkv})"
+                                   if args.shard == "heads" else
+                                   f"replicas x{world}" if world > 1 else "single GPU")},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
                      "peak_sustained": peak_sustained, "frac_sustained": achieved / peak_sustained,
@@ -380,6 +400,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with several GPUs: each runs its own replica of the workload (weak scaling), or the "
+                         "GPUs split the workload's heads (strong scaling; Hkv must divide by the GPU count)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="host time for the cpu_baseline sample of the CUDA arm")
     ap.add_argument("--ref-seconds", type=float, default=150.0,

@@ -131,3 +131,31 @@ def sample_rows(N: int, window: int, count: int, seed: int):
             if 0 <= r < N:
                 rows.add(r)
     return sorted(rows)
+
+
+def head_shard(w: Workload, world: int, rank: int):
+    """Head-sharded multi-GPU layout: rank `rank` of `world` owns the
+    contiguous block of KV heads [kv_lo, kv_hi) and their query heads
+    [kv_lo * g, kv_hi * g) (g = Hq / Hkv), as a tensor-parallel model holds
+    its own heads.  (b, h) problems are independent, so no data moves
+    between ranks.  Returns (sub-workload, q_lo, q_hi, kv_lo, kv_hi)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("need 0 <= rank < world")
+    if w.Hkv % world != 0:
+        raise ValueError(f"Hkv={w.Hkv} is not divisible by {world} ranks")
+    per = w.Hkv // world
+    kv_lo, kv_hi = rank * per, (rank + 1) * per
+    q_lo, q_hi = kv_lo * w.group, kv_hi * w.group
+    sub = dataclasses.replace(w, name=f"{w.name}_heads{rank}of{world}", Hq=q_hi - q_lo, Hkv=per)
+    return sub, q_lo, q_hi, kv_lo, kv_hi
+
+
+def shard_inputs(inp: Dict[str, Optional[torch.Tensor]], q_lo: int, q_hi: int, kv_lo: int, kv_hi: int):
+    """This rank's contiguous slices of a workload's inputs (and per-head
+    scales) along the head dimension."""
+    out: Dict[str, Optional[torch.Tensor]] = {}
+    for name, (lo, hi) in (("q", (q_lo, q_hi)), ("k", (kv_lo, kv_hi)), ("v", (kv_lo, kv_hi))):
+        out[name] = inp[name][:, :, lo:hi, :].contiguous()
+        s = inp[name + "_scale"]
+        out[name + "_scale"] = None if s is None else s[lo:hi].contiguous()
+    return out

@@ -7,6 +7,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -73,3 +74,92 @@ def test_reference_arm_other_ranks_exit_without_work():
            "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
     proc = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert proc.returncode == 0 and proc.stdout.strip() == ""
+
+
+# ---- head-sharded multi-GPU layout (each rank owns a block of KV heads and
+# their query heads; no data moves between ranks)
+
+from exact_io_aware_78_b200 import accounting  # noqa: E402
+from exact_io_aware_78_b200.inputs import WORKLOADS, head_shard, make_inputs, shard_inputs  # noqa: E402
+from dataclasses import replace as dataclasses_replace  # noqa: E402
+
+
+@pytest.mark.parametrize("name", ["bf16_causal_b4h16_n2048_d128", "bf16_gqa_causal_b2h32kv8_n4096_d128_q3",
+                                  "fp8_causal_b2h16_n8192_d128"])
+@pytest.mark.parametrize("world", [1, 2, 4, 8])
+def test_head_shards_partition_the_heads(name, world):
+    w = WORKLOADS[name]
+    q_seen, kv_seen, flops = [], [], 0.0
+    for rank in range(world):
+        sub, q_lo, q_hi, kv_lo, kv_hi = head_shard(w, world, rank)
+        q_seen += list(range(q_lo, q_hi))
+        kv_seen += list(range(kv_lo, kv_hi))
+        # every query head of the shard reads a KV head of the same shard
+        assert all(kv_lo <= h // w.group < kv_hi for h in range(q_lo, q_hi))
+        assert sub.group == w.group and sub.Hq == q_hi - q_lo and sub.Hkv == kv_hi - kv_lo
+        flops += accounting.flops(sub)
+    assert q_seen == list(range(w.Hq)) and kv_seen == list(range(w.Hkv))
+    assert flops == pytest.approx(accounting.flops(w))
+
+
+def test_head_shard_rejects_uneven_splits():
+    with pytest.raises(ValueError):
+        head_shard(WORKLOADS["bf16_gqa_causal_b2h32kv8_n4096_d128_q3"], 3, 0)
+    with pytest.raises(ValueError):
+        head_shard(WORKLOADS["bf16_causal_b4h16_n2048_d128"], 2, 2)
+
+
+def test_sharded_results_are_the_full_results():
+    """Attention per (b, h) involves no other head, so the oracle run on each
+    shard's slices and concatenated along the heads equals the oracle on the
+    whole problem (GQA, e4m3 scales included)."""
+    import oracle
+    w = dataclasses_replace(WORKLOADS["fp8_causal_b2h16_n8192_d128"], B=1, Hq=4, Hkv=2, N=40, d=128)
+    inp = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, 77)
+
+    def run(x):
+        q, k, v = (oracle.dequantize_per_head(x[n].view(torch.uint8).numpy(), x[n + "_scale"].numpy())
+                   for n in "qkv")
+        return oracle.attention_ref(q, k, v, w.causal, w.window, w.scale)
+
+    full_o, full_l = run(inp)
+    parts = []
+    for rank in range(2):
+        _, q_lo, q_hi, kv_lo, kv_hi = head_shard(w, 2, rank)
+        parts.append(run(shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)))
+    o = np.concatenate([p[0] for p in parts], axis=2)
+    l = np.concatenate([p[1] for p in parts], axis=1)
+    assert np.array_equal(o, full_o) and np.array_equal(l, full_l)
+
+
+def test_sharded_tflops_is_strong_scaling_over_the_slowest_rank():
+    # the whole problem (1e12 FLOP per step) x 10 steps in 4 ms (slowest rank)
+    assert bench.sharded_tflops(1e12, 10, 4.0) == pytest.approx(2500.0)
+
+
+def _shard_rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = WORKLOADS["bf16_gqa_causal_b2h32kv8_n4096_d128_q3"]
+        sub, q_lo, q_hi, kv_lo, kv_hi = head_shard(w, world, rank)
+        f = torch.tensor([accounting.flops(sub)], dtype=torch.float64)
+        dist.all_reduce(f)
+        slowest = bench.dist_max(2.0 + rank, world, torch.device("cpu"))
+        out[rank] = (q_lo, q_hi, float(f.item()), bench.sharded_tflops(accounting.flops(w), 10, slowest))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_shards_over_two_gloo_ranks():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_shard_rank_main, args=(world, _free_port(), out), nprocs=world, join=True,
+                       start_method="spawn")
+    w = WORKLOADS["bf16_gqa_causal_b2h32kv8_n4096_d128_q3"]
+    total = accounting.flops(w)
+    assert out[0][:2] == (0, 16) and out[1][:2] == (16, 32)
+    for rank in range(world):
+        assert out[rank][2] == pytest.approx(total)
+        assert out[rank][3] == pytest.approx(total * 10 / 3e-3 / 1e12)  # slowest rank: 3 ms
