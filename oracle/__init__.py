@@ -5,6 +5,7 @@ import this package.  It shares no code with the CUDA path.
 """
 from .attention import (allowed_mask, attention_ref, decode_e4m3, dequantize_per_head,
                         online_ref, probabilities_ref)
+from .decode import attention_kv_ref, merge_partials_ref
 
-__all__ = ["allowed_mask", "attention_ref", "decode_e4m3", "dequantize_per_head",
-           "online_ref", "probabilities_ref"]
+__all__ = ["allowed_mask", "attention_kv_ref", "attention_ref", "decode_e4m3", "dequantize_per_head",
+           "merge_partials_ref", "online_ref", "probabilities_ref"]
