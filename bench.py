@@ -30,13 +30,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_78_b200 import accounting  # noqa: E402
-from exact_io_aware_78_b200.inputs import (DEFAULT_BENCH_WORKLOAD, WORKLOADS, head_shard,  # noqa: E402
-                                           shard_inputs, workload_inputs)
+from exact_io_aware_78_b200.inputs import (DECODE_WORKLOADS, DEFAULT_BENCH_WORKLOAD, WORKLOADS,  # noqa: E402
+                                           decode_workload_inputs, head_shard, shard_inputs, workload_inputs)
 
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh",
-                  "exact_io_aware_78_b200/csrc/exactattn.cu"]
+KERNEL_SOURCES = ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_kernel.cuh",
+                  "exact_io_aware_78_b200/csrc/sm100_ptx.cuh", "exact_io_aware_78_b200/csrc/exactattn.cu"]
 
 
 def kernel_source_hash() -> str:
@@ -219,6 +219,43 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+class DecodeOracleSampler:
+    """Times the float64 decode oracle one (b, h) head at a time (its Nq
+    query rows against the whole cache), continuing where it stopped."""
+
+    def __init__(self, w):
+        inp = decode_workload_inputs(w)
+        self.w = w
+        self.qkv = [inp[n].to(torch.float64).numpy() for n in "qkv"]
+        self.cursor = 0
+
+    def run(self, budget_s: float):
+        """Returns (seconds, attended FLOPs covered, query rows done)."""
+        from oracle import attention_kv_ref  # CPU baseline leg only
+
+        w = self.w
+        q, k, v = self.qkv
+        pairs = accounting.decode_pairs(w.Nq, w.Nk, w.causal, w.window)
+        flops = 0.0
+        rows_done = 0
+        t0 = time.perf_counter()
+        while True:
+            b, h = divmod(self.cursor % (w.B * w.Hq), w.Hq)
+            self.cursor += 1
+            kh = h // w.group
+            attention_kv_ref(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, kh:kh + 1], v[b:b + 1, :, kh:kh + 1],
+                             w.causal, w.window, w.scale)
+            flops += 4.0 * w.d * pairs
+            rows_done += w.Nq
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        return time.perf_counter() - t0, flops, rows_done
+
+
+def is_decode(w) -> bool:
+    return w.name in DECODE_WORKLOADS
+
+
 def run_reference(args, w, world, rank):
     if rank != 0:
         return
@@ -226,7 +263,7 @@ def run_reference(args, w, world, rank):
     flops_done = 0.0
     rows_total = 0
     per_step_budget = min(20.0, args.ref_seconds / max(1, args.steps + args.warmup))
-    sampler = OracleSampler(w)
+    sampler = DecodeOracleSampler(w) if is_decode(w) else OracleSampler(w)
     for i in range(args.warmup + args.steps):
         dt, fl, rows = sampler.run(per_step_budget)
         if i >= args.warmup:
@@ -234,20 +271,29 @@ def run_reference(args, w, world, rank):
             flops_done += fl
             rows_total += rows
     value = flops_done / sum(times) / 1e12
-    sample = (f"{rows_total} query rows (128-row chunks of consecutive (b,h) heads) of {w.name} over "
+    unit_desc = ("query rows (all Nq rows of consecutive (b,h) heads)" if is_decode(w) else
+                 "query rows (128-row chunks of consecutive (b,h) heads)")
+    sample = (f"{rows_total} {unit_desc} of {w.name} over "
               f"{args.steps} steps of ~{per_step_budget:.3g} s, numpy float64 two-pass oracle; "
               f"TFLOP/s counts attended-pair FLOPs")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-                   "causal": w.causal, "window": w.window, "input_dtype": w.dtype},
+        "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def workload_config(w) -> dict:
+    if is_decode(w):
+        return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                "causal": w.causal, "window": w.window, "input_dtype": "bf16"}
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "causal": w.causal, "window": w.window, "input_dtype": w.dtype}
 
 
 # ------------------------------------------------------------- CUDA arm
@@ -393,12 +439,134 @@ def run_cuda(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_cuda(args, w, world, rank, local):
+    """A decode step (attn_fwd_decode): Nq new query rows per (b, h) against a
+    cache of Nk keys.  HBM-bound, so the roofline is the measured copy
+    bandwidth over the step's algorithmic bytes (Q, the visible K/V rows, O,
+    LSE, each moved once); the value is still attended-pair TFLOP/s."""
+    import exact_io_aware_78_b200 as ea
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    w_job = w
+    inp = decode_workload_inputs(w)
+    if args.shard == "heads":
+        w, q_lo, q_hi, kv_lo, kv_hi = head_shard(w_job, world, rank)
+        inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    o = torch.empty((w.B, w.Nq, w.Hq, w.d), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((w.B, w.Hq, w.Nq), device=dev, dtype=torch.float32)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_fwd_decode(q, k, v, o, lse, w.causal, w.window, w.scale, 0, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    step_ms = [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
+    total_ms = dist_max(sum(step_ms), world, dev)
+    flops = accounting.decode_flops(w)
+    if args.shard == "heads":
+        value = sharded_tflops(accounting.decode_flops(w_job), args.steps, total_ms)
+    else:
+        value = job_tflops(flops, args.steps, world, total_ms)
+
+    # e2e: the public call with the step's inputs copied from pinned host memory
+    qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    es = torch.cuda.Event(enable_timing=True)
+    ee = torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(e2e_steps + 2):
+        flush.zero_()
+        es.record(stream)
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+        ee.record(stream)
+        ee.synchronize()
+        if i >= 2:
+            e2e_ms.append(es.elapsed_time(ee))
+    e2e_total = dist_max(sum(e2e_ms), world, dev)
+    if args.shard == "heads":
+        e2e_value = sharded_tflops(accounting.decode_flops(w_job), e2e_steps, e2e_total)
+    else:
+        e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    launch_ms = statistics.mean(step_ms)
+    nbytes = accounting.decode_bytes(w)
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "strong" if args.shard == "heads" else "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(workload_config(w_job), flops_per_step=accounting.decode_flops(w_job),
+                       l2="flushed between timed steps (256 MiB write, untimed)",
+                       parallelism=(f"head shards x{world}" if args.shard == "heads" else
+                                    f"replicas x{world}" if world > 1 else "single GPU")),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": load_traffic(w.name),
+                     "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes": nbytes,
+                     "kernel_source_hash": kernel_source_hash()},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 2,  # key-range kernel + combine kernel
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        dt, fl, rows = DecodeOracleSampler(w).run(args.cpu_seconds)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"{rows} query rows (all Nq rows of consecutive (b,h) heads) of "
+                                          f"{w.name} in {dt:.1f} s, numpy float64 two-pass oracle; TFLOP/s "
+                                          f"counts attended-pair FLOPs"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="with several GPUs: each runs its own replica of the workload (weak scaling), or the "
@@ -411,14 +579,14 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = WORKLOADS[args.workload]
+    w = WORKLOADS[args.workload] if args.workload in WORKLOADS else DECODE_WORKLOADS[args.workload]
     if args.impl == "reference":
         # host-only: rank 0 times the oracle, other ranks exit without work
         run_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
     world, rank, local = init_dist()
     try:
-        run_cuda(args, w, world, rank, local)
+        (run_decode_cuda if is_decode(w) else run_cuda)(args, w, world, rank, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -37,6 +37,10 @@ _SIGNATURES = {
                                              ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]),
+    "attn_fwd_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
 }
 
 _lib = None
@@ -139,6 +143,54 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
                     dtype=torch.float32 if q.dtype == torch.float32 else torch.bfloat16)
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
     attn_fwd(q, k, v, o, lse, causal, window, scale, q_scale, k_scale, v_scale, stream)
+    return o, lse
+
+
+def attn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                    causal: bool = True, window: int = 0, scale: Optional[float] = None, num_splits: int = 0,
+                    stream=None) -> None:
+    """Queue O, LSE for Nq new query rows against Nk >= Nq cached keys on
+    `stream`.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], o [B,Nq,Hq,d] bf16,
+    lse [B,Hq,Nq] fp32, contiguous CUDA tensors on one device; query row i is
+    the token at position Nk - Nq + i."""
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, N, H, d]")
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
+        raise ValueError("q, k, v, o must be bfloat16")
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Nk, Hkv, d) or tuple(v.shape) != (B, Nk, Hkv, d):
+        raise ValueError("k and v must be [B, Nk, Hkv, d] matching q")
+    if tuple(o.shape) != (B, Nq, Hq, d):
+        raise ValueError("o must be [B, Nq, Hq, d]")
+    if tuple(lse.shape) != (B, Hq, Nq) or lse.dtype != torch.float32:
+        raise ValueError("lse must be [B, Hq, Nq] float32")
+    if len({t.device for t in (q, k, v, o, lse)}) != 1:
+        raise ValueError("all tensors must be on one device")
+    if scale is None:
+        scale = d ** -0.5
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq,
+                                 Hkv, Nq, Nk, d, int(bool(causal)), int(window), float(scale), EA_BF16,
+                                 int(num_splits), _stream_handle(stream, q.device))
+    if st != EA_OK:
+        raise AttnError(st, "attn_fwd_decode")
+
+
+def forward_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, window: int = 0,
+                   scale: Optional[float] = None, num_splits: int = 0,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Allocate O and LSE on q's device and run attn_fwd_decode."""
+    B, Nq, Hq, d = q.shape
+    o = torch.empty((B, Nq, Hq, d), device=q.device, dtype=torch.bfloat16)
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
+    attn_fwd_decode(q, k, v, o, lse, causal, window, scale, num_splits, stream)
     return o, lse
 
 

@@ -57,3 +57,30 @@ def algorithmic_bytes(w: Workload) -> int:
     lse = w.B * w.Hq * w.N * 4
     scales = (w.Hq + 2 * w.Hkv) * 4 if w.dtype == "fp8" else 0
     return q + kv + o + lse + scales
+
+
+def decode_pairs(Nq: int, Nk: int, causal: bool, window: int) -> int:
+    """Attended (query, key) pairs of one (b, h) in a decode step: query i
+    sits at position Nk - Nq + i."""
+    total = 0
+    for i in range(Nq):
+        pos = Nk - Nq + i
+        hi = pos + 1 if causal else Nk
+        lo = max(0, pos - window + 1) if window > 0 else 0
+        total += max(0, hi - lo)
+    return total
+
+
+def decode_flops(w) -> float:
+    """4 * d FLOPs per attended pair, over B * Hq."""
+    return 4.0 * w.d * w.B * w.Hq * decode_pairs(w.Nq, w.Nk, w.causal, w.window)
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic bytes of a decode step: Q read once, the K and V rows some
+    query can see read once (with a window, only the last window + Nq - 1),
+    O and LSE written once (bf16, LSE fp32)."""
+    key_lo = max(0, w.Nk - w.Nq - w.window + 1) if w.window > 0 else 0
+    q = w.B * w.Nq * w.Hq * w.d * 2
+    kv = 2 * w.B * (w.Nk - key_lo) * w.Hkv * w.d * 2
+    return q + kv + q + w.B * w.Hq * w.Nq * 4

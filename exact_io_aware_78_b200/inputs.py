@@ -159,3 +159,54 @@ def shard_inputs(inp: Dict[str, Optional[torch.Tensor]], q_lo: int, q_hi: int, k
         s = inp[name + "_scale"]
         out[name + "_scale"] = None if s is None else s[lo:hi].contiguous()
     return out
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """A decode step: Nq new query rows (the last tokens of the sequence)
+    against a key/value cache of Nk rows; bf16 inputs."""
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    window: int
+    seed: int
+    description: str = ""
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+
+DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
+    w.name: w
+    for w in [
+        DecodeWorkload("decode_b8h32kv8_nq1_nk16384_d128", 8, 32, 8, 1, 16384, 128, True, 0, 1601,
+                       description="one new token per sequence, GQA 4:1, 16384-token cache"),
+        DecodeWorkload("decode_b4h32kv8_nq2_nk8192_d128_window2048", 4, 32, 8, 2, 8192, 128, True, 2048, 1602,
+                       description="two new tokens, causal within the step, sliding window 2048"),
+    ]
+}
+
+
+def make_decode_inputs(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int,
+                       seed: int) -> Dict[str, Optional[torch.Tensor]]:
+    """Q [B, Nq, Hq, d], K, V [B, Nk, Hkv, d]: seeded N(0, 1) on the CPU
+    (seeds seed, seed+1, seed+2), stored as bf16 (no per-head scales)."""
+    return {"q": _randn(seed + 0, (B, Nq, Hq, d)).to(torch.bfloat16),
+            "k": _randn(seed + 1, (B, Nk, Hkv, d)).to(torch.bfloat16),
+            "v": _randn(seed + 2, (B, Nk, Hkv, d)).to(torch.bfloat16),
+            "q_scale": None, "k_scale": None, "v_scale": None}
+
+
+def decode_workload_inputs(w: DecodeWorkload) -> Dict[str, Optional[torch.Tensor]]:
+    return make_decode_inputs(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.seed)

@@ -173,6 +173,46 @@ int attn_version(void);
 int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq,
                           int Hkv, int N, int d, int causal, int window, float scale, int* status, void* stream);
 
+/*
+ * attn_fwd_decode -- the same exact attention for Nq new query rows against a
+ * key/value cache of Nk >= Nq rows (a decode step), computed by splitting the
+ * keys across warps and merging the parts' results with their log-sum-exps.
+ *
+ * What it computes: the pages' softmax(scale Q K^T + mask) V with its
+ * per-row log-sum-exp ("Flash Attention" concept note, AS-IS diagram; Hacker
+ * News discussion, item 40939398), key blocks combined through their
+ * normalisation factors ("Flash Attention" note, TO-BE diagram and "Tiling"
+ * section), split across parallel workers as in the decoding work the pages
+ * list by title (FlashDecoding++).  Query row i is the token at position
+ * Nk - Nq + i (the new tokens end the sequence): with causal = 1 it sees keys
+ * 0 .. Nk - Nq + i; with window > 0 only keys j > Nk - Nq + i - window.
+ *
+ * Arguments and layout (all device pointers, d contiguous, caller-owned):
+ *   q    [B, Nq, Hq, d]  bf16        o    [B, Nq, Hq, d]  bf16 (written)
+ *   k, v [B, Nk, Hkv, d] bf16        lse  [B, Hq, Nq]     fp32 (written, natural log)
+ *   dtype must be EA_BF16; d is 64 or 128; (Hq / Hkv) * Nq <= 8 query rows
+ *   per key/value head (larger query blocks: use attn_fwd).
+ *   num_splits: key ranges per (batch, key/value head); 0 chooses enough for
+ *   about 16 warps per SM.  Results for different split counts agree within
+ *   rounding; a given split count is deterministic.
+ *   stream: cudaStream_t (NULL = default stream); the call is asynchronous.
+ *
+ * Memory: the partial results (per range and query row: 2 + d floats) come
+ * stream-ordered from the library's memory pool and go back to it on the
+ * stream; attn_shutdown() releases the pool.
+ *
+ * Errors (returned synchronously, nothing queued): EA_EINVAL for NULL
+ * pointers, non-positive sizes, Nq > Nk, Hq not a multiple of Hkv, causal not
+ * 0/1, a non-positive or non-finite scale, an unknown dtype, negative
+ * num_splits, or a buffer that is not one device allocation large enough;
+ * EA_EUNSUPPORTED for fp8/fp32 inputs, d other than 64/128, or more than 8
+ * query rows per key/value head; EA_EALIGN unless q, k, v, o are 16-byte and
+ * lse 4-byte aligned; EA_ENOMEM when the pool cannot supply the partials;
+ * EA_ECUDA without a usable sm_100 device; EA_ELAUNCH if a launch fails.
+ */
+int attn_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                    int Nk, int d, int causal, int window, float scale, int dtype, int num_splits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -163,3 +163,15 @@ def test_head_shards_over_two_gloo_ranks():
     for rank in range(world):
         assert out[rank][2] == pytest.approx(total)
         assert out[rank][3] == pytest.approx(total * 10 / 3e-3 / 1e12)  # slowest rank: 3 ms
+
+
+def test_reference_arm_on_a_decode_workload():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+           "decode_b4h32kv8_nq2_nk8192_d128_window2048", "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr
+    lines = [l for l in proc.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["config"]["Nq"] == 2 and j["config"]["Nk"] == 8192
+    assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"

@@ -27,7 +27,7 @@ def lib(lib_path):
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_get_last_error", "attn_status_string", "attn_set_option", "attn_shutdown",
-         "attn_version", "attn_fwd_fp32_noalloc"])
+         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode"])
 
 
 def test_library_exports_every_declared_symbol(lib_path):
@@ -113,3 +113,41 @@ def test_python_binding_rejects_bad_layouts():
     q = torch.zeros(1, 8, 2, 64)
     with pytest.raises(ValueError):
         B.attn_fwd(q, q, q, q, torch.zeros(1, 2, 8))          # CPU tensors
+
+
+def call_decode(lib, q=P, k=P, v=P, o=P, lse=P, B_=1, Hq=8, Hkv=2, Nq=1, Nk=4096, d=128, causal=1, window=0,
+                scale=0.125, dtype=B.EA_BF16, splits=0):
+    return lib.attn_fwd_decode(q, k, v, o, lse, B_, Hq, Hkv, Nq, Nk, d, causal, window, scale, dtype, splits, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), B.EA_EINVAL),
+    (dict(Nq=0), B.EA_EINVAL),
+    (dict(Nk=0), B.EA_EINVAL),
+    (dict(Nq=5, Nk=4), B.EA_EINVAL),                     # more new queries than cached keys
+    (dict(Hq=6, Hkv=4), B.EA_EINVAL),
+    (dict(causal=3), B.EA_EINVAL),
+    (dict(scale=0.0), B.EA_EINVAL),
+    (dict(splits=-1), B.EA_EINVAL),
+    (dict(dtype=9), B.EA_EINVAL),
+    (dict(dtype=B.EA_FP8_E4M3), B.EA_EUNSUPPORTED),
+    (dict(dtype=B.EA_FP32), B.EA_EUNSUPPORTED),
+    (dict(d=96), B.EA_EUNSUPPORTED),
+    (dict(Hq=16, Hkv=2, Nq=2), B.EA_EUNSUPPORTED),       # 16 query rows per KV head > 8
+    (dict(o=P + 8), B.EA_EALIGN),
+    (dict(lse=P + 2), B.EA_EALIGN),
+    (dict(), None),                                       # valid: reaches the device step
+])
+def test_decode_argument_errors(lib, kw, code):
+    rc = call_decode(lib, **kw)
+    if code is None:
+        assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
+    else:
+        assert rc == code
+
+
+def test_python_decode_binding_rejects_bad_layouts():
+    import torch
+    q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.attn_fwd_decode(q, q, q, q, torch.zeros(1, 8, 1))     # CPU tensors

@@ -77,3 +77,39 @@ def test_sample_rows_cover_edges():
     assert r == sorted(set(r))
     rw = sample_rows(16384, 4096, 16, 3)
     assert 4095 in rw and 4096 in rw
+
+
+# ---- decode steps
+
+from exact_io_aware_78_b200.accounting import decode_bytes, decode_flops, decode_pairs  # noqa: E402
+from exact_io_aware_78_b200.inputs import DECODE_WORKLOADS, make_decode_inputs  # noqa: E402
+
+
+@pytest.mark.parametrize("Nq,Nk,causal,window", [(1, 1, True, 0), (1, 100, True, 0), (3, 100, True, 0),
+                                                  (3, 100, False, 0), (4, 50, True, 7), (2, 9, False, 3),
+                                                  (5, 5, True, 0)])
+def test_decode_pairs_by_brute_force(Nq, Nk, causal, window):
+    n = 0
+    for i in range(Nq):
+        pos = Nk - Nq + i
+        for j in range(Nk):
+            if (not causal or j <= pos) and (window <= 0 or j > pos - window):
+                n += 1
+    assert decode_pairs(Nq, Nk, causal, window) == n
+
+
+def test_decode_workload_accounting():
+    w = DECODE_WORKLOADS["decode_b8h32kv8_nq1_nk16384_d128"]
+    assert decode_flops(w) == 4 * 128 * 8 * 32 * 16384
+    # K and V of every cached row read once dominate the bytes
+    assert decode_bytes(w) == 2 * 8 * 1 * 32 * 128 * 2 + 2 * 8 * 16384 * 8 * 128 * 2 + 8 * 32 * 4
+    ww = DECODE_WORKLOADS["decode_b4h32kv8_nq2_nk8192_d128_window2048"]
+    # only the last window + Nq - 1 keys can be seen
+    assert decode_bytes(ww) == 2 * 4 * 2 * 32 * 128 * 2 + 2 * 4 * (2048 + 1) * 8 * 128 * 2 + 4 * 32 * 2 * 4
+
+
+def test_decode_inputs_are_seeded_bf16():
+    a = make_decode_inputs(2, 4, 2, 1, 33, 64, seed=3)
+    b = make_decode_inputs(2, 4, 2, 1, 33, 64, seed=3)
+    assert all(torch.equal(a[n], b[n]) for n in "qkv")
+    assert a["q"].shape == (2, 1, 4, 64) and a["k"].shape == (2, 33, 2, 64) and a["q"].dtype == torch.bfloat16
