@@ -35,13 +35,19 @@ from exact_io_aware_78_b200.inputs import (DECODE_WORKLOADS, DEFAULT_BENCH_WORKL
 
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_kernel.cuh",
-                  "exact_io_aware_78_b200/csrc/sm100_ptx.cuh", "exact_io_aware_78_b200/csrc/exactattn.cu"]
+# The sources behind each kind of workload's kernels and launch code; a
+# recorded ncu traffic figure is valid only while their hash is unchanged.
+KERNEL_SOURCES = {
+    "prefill": ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh",
+                "exact_io_aware_78_b200/csrc/exactattn.cu"],
+    "decode": ["exact_io_aware_78_b200/csrc/decode_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_api.cuh",
+               "exact_io_aware_78_b200/csrc/sm100_ptx.cuh"],
+}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kind: str = "prefill") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -64,7 +70,8 @@ def load_traffic(workload: str):
     with open(path) as f:
         data = json.load(f)
     ent = data.get(workload)
-    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+    kind = "decode" if workload.startswith("decode_") else "prefill"
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash(kind):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -546,7 +553,7 @@ def run_decode_cuda(args, w, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": load_traffic(w.name),
                      "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes": nbytes,
-                     "kernel_source_hash": kernel_source_hash()},
+                     "kernel_source_hash": kernel_source_hash("decode")},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * 2,  # key-range kernel + combine kernel
         "clocks": clocks,

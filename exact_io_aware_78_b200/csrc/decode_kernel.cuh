@@ -63,6 +63,16 @@ struct DecodeParams {
   float scale_log2; // scale * log2(e)
 };
 
+// 16-byte asynchronous global->shared copy; src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -77,12 +87,20 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
   const long long task = static_cast<long long>(blockIdx.x) * kDecodeWarps + warp;
   const long long tasks = static_cast<long long>(p.B) * p.Hkv * p.splits;
   if (task >= tasks) return;  // whole warp
-  const int split = static_cast<int>(task % p.splits);
-  const int bk = static_cast<int>(task / p.splits);  // b * Hkv + hkv
-  const int b = bk / p.Hkv, hkv = bk - b * p.Hkv;
+  // Consecutive warps take consecutive kv heads of the same batch and key
+  // range, so a block reads neighbouring 2*d-byte pieces of the same key
+  // rows (a key row of all heads is contiguous) at about the same time.
+  const int hkv = static_cast<int>(task % p.Hkv);
+  const int split = static_cast<int>((task / p.Hkv) % p.splits);
+  const int b = static_cast<int>(task / (static_cast<long long>(p.Hkv) * p.splits));
+  const int bk = b * p.Hkv + hkv;
+  const long long part = static_cast<long long>(bk) * p.splits + split;  // partial-result slot
   const int R = p.rows;
-  float* qs = dec_smem + warp * (kRows * kD + 32 * kRows);
+  constexpr int kRowBytes = kD * 2 + 16;  // a staged K row, padded so lanes reading rows hit distinct banks
+  constexpr int kWarpFloats = kRows * kD + 32 * kRows + 2 * 32 * kRowBytes / 4;
+  float* qs = dec_smem + warp * kWarpFloats;
   float* ps = qs + kRows * kD;
+  uint8_t* kbuf = reinterpret_cast<uint8_t*>(ps + 32 * kRows);  // two batches of 32 K rows
 
   // Stage this group's query rows (row r = head-in-group * Nq + i), scaled;
   // rows past R are zero.
@@ -118,21 +136,26 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
   // its scores are computed, and the next batch's K rows before its P V, so
   // each load's latency overlaps compute.
   using VSlice = typename std::conditional<kPerLane == 4, uint2, uint32_t>::type;
-  uint4 kw[kD / 8];
-  auto load_k = [&](int kb) {
-    const int jj = kb + lane;
-    if (jj < k_end) {
-      const uint4* krow = reinterpret_cast<const uint4*>(kbase + static_cast<size_t>(jj) * row_stride);
+  // K rows of a batch are copied to shared memory by the whole warp, each
+  // instruction covering two whole rows (coalesced), one batch ahead.
+  constexpr int kChunks = kD * 2 / 16;  // 16-byte chunks per row
+  auto load_k = [&](int kb, int buf) {
+    uint8_t* dst = kbuf + buf * 32 * kRowBytes;
 #pragma unroll
-      for (int c = 0; c < kD / 8; ++c) kw[c] = __ldg(krow + c);
-    } else {
-#pragma unroll
-      for (int c = 0; c < kD / 8; ++c) kw[c] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kChunks; ++i) {
+      const int c = i * 32 + lane;
+      const int row = c / kChunks, col = c - row * kChunks;
+      const int jj = kb + row;
+      const int js = jj < k_end ? jj : k_end - 1;  // a valid address; no bytes read past the range
+      cp_async16(dst + row * kRowBytes + col * 16, kbase + static_cast<size_t>(js) * row_stride + col * 8,
+                 jj < k_end ? 16u : 0u);
     }
+    cp_async_commit();
   };
-  if (k_begin < k_end) load_k(k_begin);
+  if (k_begin < k_end) load_k(k_begin, 0);
 
-  for (int kb = k_begin; kb < k_end; kb += 32) {
+  int buf = 0;
+  for (int kb = k_begin; kb < k_end; kb += 32, buf ^= 1) {
     const int j = kb + lane;  // this lane's key
     const bool have = j < k_end;
     const int nk = min(32, k_end - kb);
@@ -145,6 +168,14 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
       else
         vw[t] = VSlice{};
     }
+    if (kb + 32 < k_end) {
+      load_k(kb + 32, buf ^ 1);
+      cp_async_wait<1>();  // this batch's rows have landed; the next batch's may still be in flight
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint4* krow = reinterpret_cast<const uint4*>(kbuf + buf * 32 * kRowBytes + lane * kRowBytes);
     // ---- scores s_r = q_r . k_j (log2 units): this lane's K row, paired FMAs
     uint64_t s2[kRows];
 #pragma unroll
@@ -152,10 +183,11 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
     {
 #pragma unroll
       for (int c = 0; c < kD / 8; ++c) {
-        const uint64_t k0 = f2_pack(bf16_lo(kw[c].x), bf16_hi(kw[c].x));
-        const uint64_t k1 = f2_pack(bf16_lo(kw[c].y), bf16_hi(kw[c].y));
-        const uint64_t k2 = f2_pack(bf16_lo(kw[c].z), bf16_hi(kw[c].z));
-        const uint64_t k3 = f2_pack(bf16_lo(kw[c].w), bf16_hi(kw[c].w));
+        const uint4 kw = krow[c];
+        const uint64_t k0 = f2_pack(bf16_lo(kw.x), bf16_hi(kw.x));
+        const uint64_t k1 = f2_pack(bf16_lo(kw.y), bf16_hi(kw.y));
+        const uint64_t k2 = f2_pack(bf16_lo(kw.z), bf16_hi(kw.z));
+        const uint64_t k3 = f2_pack(bf16_lo(kw.w), bf16_hi(kw.w));
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
           const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + r * kD + 8 * c);
@@ -196,7 +228,6 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
 #pragma unroll
     for (int r = 0; r < kRows; ++r) ps[lane * kRows + r] = pr[r];
     __syncwarp();
-    if (kb + 32 < k_end) load_k(kb + 32);  // next batch's K rows
     // ---- O += P V over the batch: this lane's column slice of each V row
     // (the warp reads each row as one coalesced segment); keys past the
     // range have p = 0 and were not loaded
@@ -237,7 +268,7 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
     float lr = l[r];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lr += __shfl_xor_sync(0xFFFFFFFFu, lr, off);
-    const size_t pr_idx = static_cast<size_t>(task) * R + r;
+    const size_t pr_idx = static_cast<size_t>(part) * R + r;
     if (lane == 0) {
       p.part_ml[2 * pr_idx] = m[r];
       p.part_ml[2 * pr_idx + 1] = lr;
