@@ -8,7 +8,9 @@ O plus the per-row log-sum-exp written once; no N x N matrix ever moves
 """
 from __future__ import annotations
 
-from .inputs import Workload
+import numpy as np
+
+from .inputs import Workload, make_row_ranges
 
 
 def attended_pairs(N: int, causal: bool, window: int) -> int:
@@ -28,9 +30,34 @@ def attended_pairs(N: int, causal: bool, window: int) -> int:
     return w * N + tail * N - (tail * (tail + 1)) // 2
 
 
+def range_pairs(key_lo, key_hi, causal: bool, window: int) -> int:
+    """Attended pairs over all batches of per-row key ranges ([B, N] integer
+    arrays): row i sees keys [max(lo_i, 0, i - window + 1), min(hi_i, N, i + 1)),
+    the window and causal bounds applying only when set."""
+    lo = np.asarray(key_lo, dtype=np.int64)
+    hi = np.asarray(key_hi, dtype=np.int64)
+    N = lo.shape[-1]
+    i = np.arange(N, dtype=np.int64)
+    a = np.maximum(lo, 0)
+    b = np.minimum(hi, N)
+    if window > 0:
+        a = np.maximum(a, i - window + 1)
+    if causal:
+        b = np.minimum(b, i + 1)
+    return int(np.maximum(b - a, 0).sum())
+
+
+def workload_pairs(w: Workload) -> int:
+    """Attended pairs of one query head summed over the batch."""
+    if w.mask:
+        lo, hi = make_row_ranges(w.mask, w.B, w.N, w.seed + 3, w.mask_min, w.mask_max)
+        return range_pairs(lo.numpy(), hi.numpy(), w.causal, w.window)
+    return w.B * attended_pairs(w.N, w.causal, w.window)
+
+
 def flops(w: Workload) -> float:
     """4 * d FLOPs per attended pair, summed over batch and query heads."""
-    return 4.0 * w.B * w.Hq * w.d * attended_pairs(w.N, w.causal, w.window)
+    return 4.0 * w.Hq * w.d * workload_pairs(w)
 
 
 def flops_half_square(w: Workload) -> float:

@@ -35,6 +35,9 @@ class Workload:
     seed: int
     q_mult: float = 1.0  # Q drawn as q_mult * N(0, 1) before the format cast
     description: str = ""
+    mask: str = ""       # per-row key ranges: "" (none), "documents" or "prefix" (make_row_ranges)
+    mask_min: int = 0    # shortest document / prefix
+    mask_max: int = 0    # longest document / prefix
 
     @property
     def scale(self) -> float:
@@ -58,6 +61,9 @@ WORKLOADS: Dict[str, Workload] = {
                  16384, description="long context, causal + sliding window 4096"),
         Workload("fp8_causal_b2h16_n8192_d128", 2, 16, 16, 8192, 128, True, 0, "fp8", 8192,
                  description="e4m3 inputs with per-head fp32 scales"),
+        Workload("bf16_doccausal_b2h16_n16384_d128", 2, 16, 16, 16384, 128, True, 0, "bf16", 1638,
+                 description="packed documents of 512-4096 tokens, causal inside each document "
+                             "(per-row key ranges)", mask="documents", mask_min=512, mask_max=4096),
     ]
 }
 
@@ -111,7 +117,51 @@ def make_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, dtype: str, seed: int
 
 
 def workload_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
-    return make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.seed, w.q_mult)
+    out = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.seed, w.q_mult)
+    out["key_lo"] = out["key_hi"] = None
+    if w.mask:
+        out["key_lo"], out["key_hi"] = make_row_ranges(w.mask, w.B, w.N, w.seed + 3, w.mask_min, w.mask_max)
+    return out
+
+
+def make_row_ranges(kind: str, B: int, N: int, seed: int, min_len: int = 1, max_len: int = 0):
+    """Seeded per-row key ranges: int32 CPU tensors key_lo, key_hi of shape
+    [B, N] (query row i of batch b may see keys key_lo <= j < key_hi).
+
+      "documents"  the N rows are packed documents whose lengths are drawn
+                   uniformly from [min_len, max_len] (the last one cut at N);
+                   a row sees the keys of its own document.  With causal
+                   masking on top this is the packed-sequence training mask.
+      "prefix"     per batch a prefix length P drawn from [min_len, max_len]:
+                   rows i < P see keys [0, P), later rows keys [0, i]
+                   (a prefix-LM mask; use without causal masking).
+      "random"     lo drawn from [-2, N], hi = lo + a draw from [-2, N // 2]:
+                   empty rows, ranges past either end and single keys, for
+                   edge-case tests."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    lo = torch.zeros(B, N, dtype=torch.int32)
+    hi = torch.zeros(B, N, dtype=torch.int32)
+    max_len = max(max_len, min_len)
+    for b in range(B):
+        if kind == "documents":
+            start = 0
+            while start < N:
+                n = int(torch.randint(min_len, max_len + 1, (1,), generator=g))
+                end = min(N, start + n)
+                lo[b, start:end] = start
+                hi[b, start:end] = end
+                start = end
+        elif kind == "prefix":
+            P = min(N, int(torch.randint(min_len, max_len + 1, (1,), generator=g)))
+            i = torch.arange(N, dtype=torch.int32)
+            hi[b] = torch.where(i < P, torch.full_like(i, P), i + 1)
+        elif kind == "random":
+            lo[b] = torch.randint(-2, N + 1, (N,), generator=g, dtype=torch.int32)
+            hi[b] = lo[b] + torch.randint(-2, N // 2 + 1, (N,), generator=g, dtype=torch.int32)
+        else:
+            raise ValueError(f"unknown row-range kind {kind!r}")
+    return lo, hi
 
 
 def sample_rows(N: int, window: int, count: int, seed: int):

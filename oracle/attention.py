@@ -9,6 +9,7 @@ per key/value head and key/value head h // g):
 
     S[i, j]   = scale * sum_t Q[b, i, h, t] * K[b, j, h // g, t]
     allowed   = (not causal or j <= i) and (window <= 0 or j > i - window)
+                and (no row ranges or key_lo[b, i] <= j < key_hi[b, i])
     P[i, j]   = exp(S[i, j] - max_allowed S[i, :]) / sum_allowed exp(...)
     O[b,i,h]  = sum_j P[i, j] * V[b, j, h // g, :]
     LSE[b,h,i]= max_allowed S[i, :] + ln sum_allowed exp(S[i, j] - max)
@@ -25,6 +26,11 @@ Sources (the method is exact, so the oracle is the plain definition):
     approximation): same note, introduction; FlashAttention quiz
     (aiunderstanding.org), question 2; "FlashAttention-2 (PL)", opening
     paragraph.
+  * Per-row key ranges (key_lo, key_hi): the mask is the thing that decides
+    which queries see which keys (Hacker News discussion, same answer); the
+    richer masks of the FlashMask work that "FlashAttention-2 (PL)" lists
+    in its literature section are represented here by one contiguous range
+    of visible keys per query row.
   * The blockwise recurrence in `online_ref`: the note's TO-BE diagram
     (per block a partial result plus a normalisation factor) and its
     "Tiling" section (scale each block's output by the right normalisation
@@ -35,8 +41,11 @@ Readings where the pages are silent (each listed in the design notes):
   * window: a query i sees keys j with i - window < j, i.e. at most `window`
     keys ending at itself when causal; window <= 0 means no window.
   * GQA mapping: query head h uses key/value head h // (Hq / Hkv).
-  * A row with no allowed key (cannot happen with causal or no mask) gets
-    O = 0 and LSE = -inf.
+  * A row with no allowed key (cannot happen with causal or no mask; it can
+    with row ranges) gets O = 0 and LSE = -inf.
+  * Row ranges: query row i of batch b sees keys key_lo[b, i] <= j <
+    key_hi[b, i], intersected with the causal and window masks; one range
+    per row, shared by all heads; any integers (lo >= hi: no key).
   * LSE is the natural-log log-sum-exp of the scaled, masked logits.
   * e4m3 inputs enter as code * per-head scale, decoded exactly here.
 
@@ -46,7 +55,11 @@ returns that V row; causal row 0 equals V[0]; window 1 returns V row i;
 `online_ref` equals the two-pass definition on exhaustive tiny inputs;
 shift, permutation and affine invariances; the GQA reduction to repeated
 heads; hand-derived golden cases; agreement with torch's float64 scaled
-dot-product attention on CPU; e4m3 decoding against torch's cast.
+dot-product attention on CPU; e4m3 decoding against torch's cast.  Row
+ranges (tests/test_oracle_mask_pins.py): a document mask equals separate
+runs per document; ranges [i-W+1, i+1) reproduce causal + window; single
+visible key and empty rows in closed form; scalar brute force; torch SDPA
+with an explicit boolean mask; the blockwise recurrence.
 """
 from __future__ import annotations
 
@@ -96,8 +109,12 @@ def dequantize_per_head(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
 # Mask
 # --------------------------------------------------------------------------
 
-def allowed_mask(rows: Sequence[int], N: int, causal: bool, window: int) -> np.ndarray:
-    """Boolean [len(rows), N]: which keys j each query row i may attend to."""
+def allowed_mask(rows: Sequence[int], N: int, causal: bool, window: int,
+                 key_lo: Optional[np.ndarray] = None, key_hi: Optional[np.ndarray] = None) -> np.ndarray:
+    """Boolean [len(rows), N]: which keys j each query row i may attend to.
+    key_lo / key_hi, when given, are this batch's per-row bounds indexed by
+    the absolute row number (length >= max(rows) + 1): row i then also needs
+    key_lo[i] <= j < key_hi[i]."""
     i = np.asarray(rows, dtype=np.int64).reshape(-1, 1)
     j = np.arange(N, dtype=np.int64).reshape(1, -1)
     ok = np.ones((i.shape[0], N), dtype=bool)
@@ -105,6 +122,10 @@ def allowed_mask(rows: Sequence[int], N: int, causal: bool, window: int) -> np.n
         ok &= j <= i
     if window > 0:
         ok &= j > i - window
+    if key_lo is not None:
+        lo = np.asarray(key_lo, dtype=np.int64)[i[:, 0]].reshape(-1, 1)
+        hi = np.asarray(key_hi, dtype=np.int64)[i[:, 0]].reshape(-1, 1)
+        ok &= (j >= lo) & (j < hi)
     return ok
 
 
@@ -128,17 +149,32 @@ def _check_shapes(q, k, v):
     return B, N, Hq, Hkv, d
 
 
+def _check_ranges(key_lo, key_hi, B, N):
+    if (key_lo is None) != (key_hi is None):
+        raise ValueError("key_lo and key_hi come together")
+    if key_lo is None:
+        return None, None
+    lo = np.asarray(key_lo)
+    hi = np.asarray(key_hi)
+    if lo.shape != (B, N) or hi.shape != (B, N):
+        raise ValueError("key_lo, key_hi must be [B, N]")
+    if not (np.issubdtype(lo.dtype, np.integer) and np.issubdtype(hi.dtype, np.integer)):
+        raise ValueError("key ranges are integers")
+    return lo.astype(np.int64), hi.astype(np.int64)
+
+
 # --------------------------------------------------------------------------
 # Two-pass definition
 # --------------------------------------------------------------------------
 
 def _row_block(qb: np.ndarray, kb: np.ndarray, vb: np.ndarray, rows: np.ndarray,
-               causal: bool, window: int, scale: float):
+               causal: bool, window: int, scale: float, lo=None, hi=None):
     """Plain definition for one (b, h) and a set of query rows.
-    qb [R, d] holds those rows of Q; kb, vb are [N, d]."""
+    qb [R, d] holds those rows of Q; kb, vb are [N, d]; lo, hi are this
+    batch's per-row key ranges (or None)."""
     N = kb.shape[0]
     s = scale * (qb @ kb.T)                       # S = scale * Q K^T
-    ok = allowed_mask(rows, N, causal, window)
+    ok = allowed_mask(rows, N, causal, window, lo, hi)
     s_masked = np.where(ok, s, -np.inf)
     m = s_masked.max(axis=1, keepdims=True, initial=-np.inf)  # row max, allowed keys
     any_ok = ok.any(axis=1, keepdims=True)
@@ -155,18 +191,21 @@ def _row_block(qb: np.ndarray, kb: np.ndarray, vb: np.ndarray, rows: np.ndarray,
 def attention_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool = False,
                   window: int = 0, scale: Optional[float] = None,
                   rows: Optional[Sequence[int]] = None,
-                  row_chunk: int = 512) -> Tuple[np.ndarray, np.ndarray]:
+                  row_chunk: int = 512, key_lo: Optional[np.ndarray] = None,
+                  key_hi: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Exact attention forward in float64.
 
     q [B, N, Hq, d], k [B, N, Hkv, d], v [B, N, Hkv, dv] (any real dtype,
     upcast to float64).  Returns O [B, R, Hq, dv] and LSE [B, Hq, R] where R
     is N, or len(rows) when `rows` selects a subset of query rows (for
-    sampled checks at full size).  Work is chunked over rows to bound memory;
-    each chunk is still the two-pass definition."""
+    sampled checks at full size).  key_lo, key_hi: optional integer [B, N]
+    per-row key ranges (both or neither).  Work is chunked over rows to bound
+    memory; each chunk is still the two-pass definition."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     B, N, Hq, Hkv, d = _check_shapes(q, k, v)
+    key_lo, key_hi = _check_ranges(key_lo, key_hi, B, N)
     g = Hq // Hkv
     if scale is None:
         scale = 1.0 / np.sqrt(d)
@@ -181,19 +220,23 @@ def attention_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool = Fa
             vb = v[b, :, kv_head_of(h, Hq, Hkv), :]
             for c0 in range(0, R, row_chunk):
                 r = sel[c0:c0 + row_chunk]
-                o, l, _ = _row_block(q[b, r, h, :], kb, vb, r, causal, window, scale)
+                o, l, _ = _row_block(q[b, r, h, :], kb, vb, r, causal, window, scale,
+                                     None if key_lo is None else key_lo[b],
+                                     None if key_hi is None else key_hi[b])
                 out[b, c0:c0 + r.shape[0], h, :] = o
                 lse[b, h, c0:c0 + r.shape[0]] = l
     return out, lse
 
 
 def probabilities_ref(q: np.ndarray, k: np.ndarray, causal: bool = False, window: int = 0,
-                      scale: Optional[float] = None) -> np.ndarray:
+                      scale: Optional[float] = None, key_lo: Optional[np.ndarray] = None,
+                      key_hi: Optional[np.ndarray] = None) -> np.ndarray:
     """The full probability matrix P [B, Hq, N, N] (small inputs only)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
+    key_lo, key_hi = _check_ranges(key_lo, key_hi, B, N)
     g = Hq // Hkv
     if scale is None:
         scale = 1.0 / np.sqrt(d)
@@ -202,7 +245,9 @@ def probabilities_ref(q: np.ndarray, k: np.ndarray, causal: bool = False, window
     for b in range(B):
         for h in range(Hq):
             kb = k[b, :, kv_head_of(h, Hq, Hkv), :]
-            _, _, p = _row_block(q[b, :, h, :], kb, np.zeros((N, 1)), rows, causal, window, scale)
+            _, _, p = _row_block(q[b, :, h, :], kb, np.zeros((N, 1)), rows, causal, window, scale,
+                                 None if key_lo is None else key_lo[b],
+                                 None if key_hi is None else key_hi[b])
             P[b, h] = p
     return P
 
@@ -213,7 +258,8 @@ def probabilities_ref(q: np.ndarray, k: np.ndarray, causal: bool = False, window
 
 def online_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool = False,
                window: int = 0, scale: Optional[float] = None,
-               block_q: int = 1, block_k: int = 1) -> Tuple[np.ndarray, np.ndarray]:
+               block_q: int = 1, block_k: int = 1, key_lo: Optional[np.ndarray] = None,
+               key_hi: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
     """The tiled forward: for each block of query rows, walk the key/value
     blocks in order, keeping per row a running maximum m, a running
     normaliser l and an unnormalised partial output acc.  On each key block
@@ -224,6 +270,7 @@ def online_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool = False
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     B, N, Hq, Hkv, d = _check_shapes(q, k, v)
+    key_lo, key_hi = _check_ranges(key_lo, key_hi, B, N)
     g = Hq // Hkv
     dv = v.shape[3]
     if scale is None:
@@ -243,7 +290,9 @@ def online_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool = False
                 for k0 in range(0, N, block_k):
                     cols = np.arange(k0, min(N, k0 + block_k))
                     s = scale * (qi @ kb_all[cols].T)
-                    ok = allowed_mask(rows, N, causal, window)[:, cols]
+                    ok = allowed_mask(rows, N, causal, window,
+                                      None if key_lo is None else key_lo[b],
+                                      None if key_hi is None else key_hi[b])[:, cols]
                     s = np.where(ok, s, -np.inf)
                     m_new = np.maximum(m, s.max(axis=1))
                     # reference point for the exponentials: finite once any

@@ -41,7 +41,8 @@ def test_fp8_per_head_scale_definition():
 
 
 def test_workload_table():
-    assert len(WORKLOADS) == 5
+    assert len(WORKLOADS) == 6
+    assert WORKLOADS["bf16_doccausal_b2h16_n16384_d128"].mask == "documents"
     w = WORKLOADS["bf16_gqa_causal_b2h32kv8_n4096_d128_q3"]
     assert (w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, w.q_mult) == (2, 32, 8, 4096, 128, True, 3.0)
     assert w.group == 4
@@ -59,6 +60,27 @@ def test_attended_pairs_brute_force(N):
             if window > 0:
                 ok &= j > i - window
             assert accounting.attended_pairs(N, causal, window) == int(ok.sum())
+
+
+@pytest.mark.parametrize("kind", ["documents", "prefix", "random"])
+def test_range_pairs_brute_force(kind):
+    from exact_io_aware_78_b200.inputs import make_row_ranges
+    N = 50
+    lo, hi = make_row_ranges(kind, 3, N, 4, 3, 17)
+    lo, hi = lo.numpy(), hi.numpy()
+    for causal in (False, True):
+        for window in (0, 1, 6):
+            i = np.arange(N)[None, :, None]
+            j = np.arange(N)[None, None, :]
+            ok = (j >= lo[:, :, None]) & (j < hi[:, :, None])
+            if causal:
+                ok &= j <= i
+            if window > 0:
+                ok &= j > i - window
+            assert accounting.range_pairs(lo, hi, causal, window) == int(ok.sum())
+    # ranges that cover every key reduce to the mask-free count
+    full_lo, full_hi = np.zeros((2, N), np.int64), np.full((2, N), N)
+    assert accounting.range_pairs(full_lo, full_hi, True, 7) == 2 * accounting.attended_pairs(N, True, 7)
 
 
 def test_flop_counts_of_the_workloads():

@@ -226,7 +226,7 @@ def test_dequantize_per_head_broadcasts_over_heads():
 
 
 # --------------------------------------------------------- planted mistakes
-def _bad_mask_strict_causal(rows, N, causal, window):
+def _bad_mask_strict_causal(rows, N, causal, window, key_lo=None, key_hi=None):
     i = np.asarray(rows).reshape(-1, 1)
     j = np.arange(N).reshape(1, -1)
     ok = np.ones((i.shape[0], N), dtype=bool)
@@ -237,7 +237,7 @@ def _bad_mask_strict_causal(rows, N, causal, window):
     return ok
 
 
-def _bad_mask_wide_window(rows, N, causal, window):
+def _bad_mask_wide_window(rows, N, causal, window, key_lo=None, key_hi=None):
     i = np.asarray(rows).reshape(-1, 1)
     j = np.arange(N).reshape(1, -1)
     ok = np.ones((i.shape[0], N), dtype=bool)
@@ -248,26 +248,26 @@ def _bad_mask_wide_window(rows, N, causal, window):
     return ok
 
 
-def _bad_row_block_transposed_values(qb, kb, vb, rows, causal, window, scale):
-    o, lse, p = _orig_row_block(qb, kb, vb, rows, causal, window, scale)
+def _bad_row_block_transposed_values(qb, kb, vb, rows, causal, window, scale, lo=None, hi=None):
+    o, lse, p = _orig_row_block(qb, kb, vb, rows, causal, window, scale, lo, hi)
     # P^T V instead of P V (only shape-compatible when R == N)
     if p.shape[0] == p.shape[1]:
         o = p.T @ vb
     return o, lse, p
 
 
-def _bad_row_block_log2_lse(qb, kb, vb, rows, causal, window, scale):
-    o, lse, p = _orig_row_block(qb, kb, vb, rows, causal, window, scale)
+def _bad_row_block_log2_lse(qb, kb, vb, rows, causal, window, scale, lo=None, hi=None):
+    o, lse, p = _orig_row_block(qb, kb, vb, rows, causal, window, scale, lo, hi)
     return o, lse / np.log(2.0), p
 
 
-def _bad_row_block_no_scale(qb, kb, vb, rows, causal, window, scale):
-    return _orig_row_block(qb, kb, vb, rows, causal, window, 1.0)
+def _bad_row_block_no_scale(qb, kb, vb, rows, causal, window, scale, lo=None, hi=None):
+    return _orig_row_block(qb, kb, vb, rows, causal, window, 1.0, lo, hi)
 
 
-def _bad_row_block_column_softmax(qb, kb, vb, rows, causal, window, scale):
+def _bad_row_block_column_softmax(qb, kb, vb, rows, causal, window, scale, lo=None, hi=None):
     s = scale * (qb @ kb.T)
-    ok = allowed_mask(rows, kb.shape[0], causal, window)
+    ok = allowed_mask(rows, kb.shape[0], causal, window, lo, hi)
     e = np.where(ok, np.exp(s), 0.0)
     den = e.sum(axis=0, keepdims=True)   # normalised over the wrong axis
     p = np.divide(e, den, out=np.zeros_like(e), where=den > 0)
@@ -275,8 +275,8 @@ def _bad_row_block_column_softmax(qb, kb, vb, rows, causal, window, scale):
     return p @ vb, lse, p
 
 
-def _bad_row_block_negated_logits(qb, kb, vb, rows, causal, window, scale):
-    return _orig_row_block(-qb, kb, vb, rows, causal, window, scale)
+def _bad_row_block_negated_logits(qb, kb, vb, rows, causal, window, scale, lo=None, hi=None):
+    return _orig_row_block(-qb, kb, vb, rows, causal, window, scale, lo, hi)
 
 
 _orig_row_block = oa._row_block
