@@ -167,11 +167,15 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------ CPU oracle arm
-def pairs_for_rows(rows, N: int, causal: bool, window: int) -> int:
-    """Attended (query, key) pairs of the given query rows."""
+def pairs_for_rows(rows, N: int, causal: bool, window: int, key_lo=None, key_hi=None) -> int:
+    """Attended (query, key) pairs of the given query rows (key_lo, key_hi:
+    this batch's per-row key ranges, length N, or None)."""
     r = np.asarray(rows, dtype=np.int64)
     hi = np.minimum(r + 1, N) if causal else np.full_like(r, N)
     lo = np.maximum(r - window + 1, 0) if window > 0 else np.zeros_like(r)
+    if key_lo is not None:
+        lo = np.maximum(lo, np.asarray(key_lo, dtype=np.int64)[r])
+        hi = np.minimum(hi, np.asarray(key_hi, dtype=np.int64)[r])
     return int(np.maximum(hi - lo, 0).sum())
 
 
@@ -191,6 +195,7 @@ class OracleSampler:
                         for n in "qkv"]
         else:
             self.qkv = [inp[n].to(torch.float64).numpy() for n in "qkv"]
+        self.ranges = (None, None) if inp.get("key_lo") is None else (inp["key_lo"].numpy(), inp["key_hi"].numpy())
         self.cursor = 0
         self.chunks_per_head = (w.N + self.CHUNK - 1) // self.CHUNK
 
@@ -210,9 +215,14 @@ class OracleSampler:
             bh, c = divmod(idx, self.chunks_per_head)
             b, h = divmod(bh, w.Hq)
             rows = list(range(c * self.CHUNK, min(w.N, (c + 1) * self.CHUNK)))
+            lo, hi = self.ranges
+            lo_b = None if lo is None else lo[b:b + 1]
+            hi_b = None if hi is None else hi[b:b + 1]
             attention_ref(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, h // g:h // g + 1],
-                          v[b:b + 1, :, h // g:h // g + 1], w.causal, w.window, w.scale, rows=rows)
-            flops += 4.0 * w.d * pairs_for_rows(rows, w.N, w.causal, w.window)
+                          v[b:b + 1, :, h // g:h // g + 1], w.causal, w.window, w.scale, rows=rows,
+                          key_lo=lo_b, key_hi=hi_b)
+            flops += 4.0 * w.d * pairs_for_rows(rows, w.N, w.causal, w.window,
+                                                None if lo is None else lo[b], None if hi is None else hi[b])
             rows_done += len(rows)
             if time.perf_counter() - t0 >= budget_s:
                 break
@@ -299,8 +309,11 @@ def workload_config(w) -> dict:
     if is_decode(w):
         return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                 "causal": w.causal, "window": w.window, "input_dtype": "bf16"}
-    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-            "causal": w.causal, "window": w.window, "input_dtype": w.dtype}
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+           "causal": w.causal, "window": w.window, "input_dtype": w.dtype}
+    if w.mask:
+        cfg["row_ranges"] = f"{w.mask} of {w.mask_min}-{w.mask_max} tokens"
+    return cfg
 
 
 # ------------------------------------------------------------- CUDA arm
@@ -317,6 +330,8 @@ def run_cuda(args, w, world, rank, local):
         inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
     q, k, v = (inp[n].to(dev) for n in "qkv")
     scales = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
+    masked = inp.get("key_lo") is not None
+    key_lo, key_hi = (inp[n].to(dev) for n in ("key_lo", "key_hi")) if masked else (None, None)
     o_dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
     o = torch.empty((w.B, w.N, w.Hq, w.d), device=dev, dtype=o_dtype)
     lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
@@ -324,7 +339,11 @@ def run_cuda(args, w, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        ea.attn_fwd(q, k, v, o, lse, w.causal, w.window, w.scale, *scales, stream=stream)
+        if masked:
+            ea.attn_fwd_masked(q, k, v, o, lse, key_lo, key_hi, w.causal, w.window, w.scale, *scales,
+                               stream=stream)
+        else:
+            ea.attn_fwd(q, k, v, o, lse, w.causal, w.window, w.scale, *scales, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -362,6 +381,9 @@ def run_cuda(args, w, world, rank, local):
 
     # e2e: the public API with pinned host buffers, copies inside the timed region
     qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
+    host_in = [(q, qh), (k, kh), (v, vh)]
+    if masked:
+        host_in += [(key_lo, inp["key_lo"].pin_memory()), (key_hi, inp["key_hi"].pin_memory())]
     oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
@@ -371,9 +393,8 @@ def run_cuda(args, w, world, rank, local):
     for i in range(e2e_steps + 2):
         flush.zero_()
         es.record(stream)
-        q.copy_(qh, non_blocking=True)
-        k.copy_(kh, non_blocking=True)
-        v.copy_(vh, non_blocking=True)
+        for dst, src in host_in:
+            dst.copy_(src, non_blocking=True)
         step()
         oh.copy_(o, non_blocking=True)
         lh.copy_(lse, non_blocking=True)
@@ -386,7 +407,7 @@ def run_cuda(args, w, world, rank, local):
         e2e_value = sharded_tflops(accounting.flops(w_job), e2e_steps, e2e_total)
     else:
         e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    h2d = sum(src.numel() * src.element_size() for _, src in host_in)
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
 
     if rank != 0:
@@ -406,7 +427,8 @@ def run_cuda(args, w, world, rank, local):
     launch_ms = statistics.mean(step_ms)
     achieved = flops / (launch_ms * 1e-3) / 1e12
     traffic = load_traffic(w.name)
-    launches_per_step = 2 if w.dtype == "fp32" else 1  # fp32: split kernel + attention kernel
+    # fp32: + the split kernel; row ranges: + the tile-range kernel
+    launches_per_step = 1 + int(w.dtype == "fp32") + int(masked)
     line = {
         "metric": METRIC,
         "value": value,
@@ -420,8 +442,7 @@ def run_cuda(args, w, world, rank, local):
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "fp8": "e4m3", "fp32": "bf16x3 (fp32 in/out)"}[w.dtype],
         "data": "synthetic",
-        "config": {"workload": w_job.name, "B": w_job.B, "Hq": w_job.Hq, "Hkv": w_job.Hkv, "N": w_job.N,
-                   "d": w_job.d, "causal": w_job.causal, "window": w_job.window, "input_dtype": w_job.dtype,
+        "config": {**workload_config(w_job),
                    "flops_per_step": accounting.flops(w_job),
                    "flops_half_square_per_step": accounting.flops_half_square(w_job),
                    "l2": "flushed between timed steps (256 MiB write, untimed)",

@@ -27,6 +27,11 @@ _SIGNATURES = {
                                 ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "attn_fwd_masked": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_void_p]),
     "attn_get_last_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -96,6 +101,21 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     """Queue O, LSE = attention(q, k, v) on `stream` (default: the current
     stream).  q [B,N,Hq,d], k/v [B,N,Hkv,d], o [B,N,Hq,d], lse [B,Hq,N] fp32,
     all contiguous CUDA tensors on one device."""
+    _forward_call(q, k, v, o, lse, causal, window, None, None, scale, q_scale, k_scale, v_scale, stream)
+
+
+def attn_fwd_masked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                    key_lo: torch.Tensor, key_hi: torch.Tensor, causal: bool = False, window: int = 0,
+                    scale: Optional[float] = None, q_scale: Optional[torch.Tensor] = None,
+                    k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+    """attn_fwd with per-row key ranges: query row i of batch b also needs
+    key_lo[b, i] <= j < key_hi[b, i] (int32 [B, N] CUDA tensors, shared by
+    all heads)."""
+    _forward_call(q, k, v, o, lse, causal, window, key_lo, key_hi, scale, q_scale, k_scale, v_scale, stream)
+
+
+def _forward_call(q, k, v, o, lse, causal, window, key_lo, key_hi, scale, q_scale, k_scale, v_scale, stream):
     lib = load_library()
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, N, H, d]")
@@ -124,25 +144,39 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
         if t is not None and (not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    if (key_lo is None) != (key_hi is None):
+        raise ValueError("key_lo and key_hi come together")
+    for name, t in (("key_lo", key_lo), ("key_hi", key_hi)):
+        if t is not None and (not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous()
+                              or tuple(t.shape) != (B, N) or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous int32 [B, N] tensor on q's device")
     device = q.device
     with torch.cuda.device(device):
-        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                          B, Hq, Hkv, N, d, int(bool(causal)), int(window), float(scale), dtype,
-                          _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream_handle(stream, device))
+        if key_lo is None:
+            st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              B, Hq, Hkv, N, d, int(bool(causal)), int(window), float(scale), dtype,
+                              _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream_handle(stream, device))
+        else:
+            st = lib.attn_fwd_masked(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                     B, Hq, Hkv, N, d, int(bool(causal)), int(window), key_lo.data_ptr(),
+                                     key_hi.data_ptr(), float(scale), dtype, _ptr(q_scale), _ptr(k_scale),
+                                     _ptr(v_scale), _stream_handle(stream, device))
     if st != EA_OK:
-        raise AttnError(st, "attn_fwd")
+        raise AttnError(st, "attn_fwd" if key_lo is None else "attn_fwd_masked")
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, window: int = 0,
             scale: Optional[float] = None, q_scale: Optional[torch.Tensor] = None,
             k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
-            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Allocate O and LSE on q's device and run attn_fwd; returns (O, LSE)."""
+            stream=None, key_lo: Optional[torch.Tensor] = None,
+            key_hi: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Allocate O and LSE on q's device and run attn_fwd (attn_fwd_masked
+    when per-row key ranges are given); returns (O, LSE)."""
     B, N, Hq, d = q.shape
     o = torch.empty((B, N, Hq, d), device=q.device,
                     dtype=torch.float32 if q.dtype == torch.float32 else torch.bfloat16)
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
-    attn_fwd(q, k, v, o, lse, causal, window, scale, q_scale, k_scale, v_scale, stream)
+    _forward_call(q, k, v, o, lse, causal, window, key_lo, key_hi, scale, q_scale, k_scale, v_scale, stream)
     return o, lse
 
 

@@ -26,11 +26,20 @@
 //     tile max exceeds the max in use by more than kTau (log2 units), so the
 //     non-matmul work stays small ("Minimalizacja operacji nie-macierzowych").
 //   * The epilogue divides by l, converts, stores O and LSE = ln2 (m + log2 l).
+//   * Masks: causal and window masks become K/V tile ranges plus in-tile
+//     masking; per-row key ranges (one contiguous range of visible keys per
+//     query row, shared by all heads -- the mask decides which queries see
+//     which keys: Hacker News discussion, item 40939398; richer masks as in
+//     the FlashMask work listed by "FlashAttention-2 (PL)") are reduced
+//     per 128-row tile to a K/V tile range by a small pre-pass kernel, and
+//     each softmax thread masks its own row.  A tile no row of which sees a
+//     key takes no part in the pipeline and stores O = 0, LSE = -inf.
 //   * Every pipeline wait is bounded: past the time limit the thread records
 //     a timeout in the device error word, raises a CTA-wide abort flag and
 //     all roles unwind; tensor memory is released and no trap is issued.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 #include <cuda.h>
 #include <math_constants.h>
@@ -67,6 +76,11 @@ struct FwdParams {
   void* o;               // [B, N, Hq, d_out]
   float* lse;            // [B, Hq, N]
   int* err;              // device error word
+  const int* key_lo;     // [B, N] per-row key ranges, or null: row i sees keys key_lo <= j < key_hi
+  const int* key_hi;     // [B, N]
+  const int2* tile_kv;   // [B, num_qtiles] K/V tile range [x, y) of each 128-row query tile (with ranges)
+  const int* item_order; // [B * num_qblk] (batch, query block) pairs, most K/V tiles first (with ranges), or null
+  int num_qtiles;        // ceil(N / 128)
   int B, Hq, Hkv, N, group;
   int causal, window;
   float scale_log2;      // scale * log2(e)
@@ -152,8 +166,16 @@ struct TileRange {
   int active;    // tile has at least one valid query row
   int q0;        // first query row
   int last_row;  // last valid query row
-  int lo, hi;    // K/V tile range [lo, hi) this tile visits
+  int lo, hi;    // K/V tile range [lo, hi) this tile visits (empty: no row sees a key)
 };
+
+// A tile that takes part in the pipeline: it has rows and visits K/V tiles
+// (without row ranges every tile with rows does).
+template <bool kRanges>
+__device__ __forceinline__ bool live(const TileRange& r) {
+  if constexpr (kRanges) return r.active && r.lo < r.hi;
+  return r.active;
+}
 
 // The i-th work item of this CTA.  Items are ranked heaviest first (or
 // lightest first); CTAs take them in a boustrophedon order over the ranking
@@ -177,7 +199,21 @@ struct RingCursor {
   }
 };
 
+template <bool kRanges>
 __device__ __forceinline__ WorkItem decode_work(int w, const FwdParams& p) {
+  if constexpr (kRanges) {
+    // Ranked by cost: the Hq items of the pair order[w / Hq] are consecutive.
+    if (p.item_order != nullptr) {
+      WorkItem wk;
+      const int pr = w / p.Hq;
+      wk.h = w - pr * p.Hq;
+      const int pair = __ldg(p.item_order + pr);
+      wk.b = pair / p.num_qblk;
+      wk.qblk = pair - wk.b * p.num_qblk;
+      wk.hkv = wk.h / p.group;
+      return wk;
+    }
+  }
   const int bh_count = p.B * p.Hq;
   const int r = w / bh_count;
   const int bh = w - r * bh_count;
@@ -190,14 +226,23 @@ __device__ __forceinline__ WorkItem decode_work(int w, const FwdParams& p) {
 }
 
 // K/V tiles a query tile must visit: up to its last row when causal, from
-// the first key inside the first row's window when windowed.
-__device__ __forceinline__ TileRange tile_range(int qblk, int t, const FwdParams& p) {
+// the first key inside the first row's window when windowed; with per-row
+// key ranges, the span of its rows' visible keys (computed by
+// row_range_tiles_kernel before the launch).
+template <bool kRanges>
+__device__ __forceinline__ TileRange tile_range(const WorkItem& wk, int t, const FwdParams& p) {
   TileRange r;
-  r.q0 = qblk * 256 + t * 128;
+  r.q0 = wk.qblk * 256 + t * 128;
   r.active = r.q0 < p.N;
   r.last_row = min(r.q0 + 127, p.N - 1);
   if (!r.active) {
     r.lo = r.hi = 0;
+    return r;
+  }
+  if constexpr (kRanges) {
+    const int2 e = __ldg(p.tile_kv + static_cast<size_t>(wk.b) * p.num_qtiles + (r.q0 >> 7));
+    r.lo = e.x;
+    r.hi = e.y;
     return r;
   }
   const int hi_key = p.causal ? r.last_row + 1 : p.N;
@@ -241,7 +286,7 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, 
 }
 
 // ------------------------------------------------------------- TMA producer
-template <class C>
+template <class C, bool kRanges>
 __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                               const FwdParams& p, SharedCtl* ctl, uint8_t* smem) {
   const uint64_t pol_kv = l2_policy_evict_last();
@@ -255,15 +300,22 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const WorkItem wk = decode_work(w, p);
-    const TileRange r0 = tile_range(wk.qblk, 0, p);
-    const TileRange r1 = tile_range(wk.qblk, 1, p);
-    const int lo = r0.lo;
-    const int hi = r1.active ? r1.hi : r0.hi;
+    const WorkItem wk = decode_work<kRanges>(w, p);
+    const TileRange r0 = tile_range<kRanges>(wk, 0, p);
+    const TileRange r1 = tile_range<kRanges>(wk, 1, p);
+    int lo, hi;  // K/V tiles of the item: the span of both tiles' ranges
+    if constexpr (kRanges) {
+      if (!live<true>(r0) && !live<true>(r1)) continue;
+      lo = !live<true>(r1) ? r0.lo : (!live<true>(r0) ? r1.lo : min(r0.lo, r1.lo));
+      hi = !live<true>(r1) ? r0.hi : (!live<true>(r0) ? r1.hi : max(r0.hi, r1.hi));
+    } else {  // causal / window ranges grow with the query tile
+      lo = r0.lo;
+      hi = r1.active ? r1.hi : r0.hi;
+    }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const TileRange& rt = t == 0 ? r0 : r1;
-      if (!ok || !rt.active) continue;
+      if (!ok || !live<kRanges>(rt)) continue;
       ok = wait_phase(&ctl->q_empty[t], (q_iter[t] & 1u) ^ 1u, ctl, p, kSiteProdQEmpty, true);
       if (!ok) break;
       ++q_iter[t];
@@ -372,7 +424,7 @@ __device__ __forceinline__ bool settle(bool peeked, uint64_t* bar, uint32_t pari
 // the softmax's P and on O being free (tensor memory written or read by
 // other threads) are followed by tcgen05.fence::after_thread_sync; waits on
 // copies into shared memory need none.
-template <class C>
+template <class C, bool kRanges>
 __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
   constexpr uint32_t kStageUnits = C::kStageBytes >> 4;
   constexpr uint32_t kFmt = C::kEsize == 2 ? 1u : 0u;  // bf16 : e4m3
@@ -389,13 +441,23 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const WorkItem wk = decode_work(w, p);
-    const TileRange r[2] = {tile_range(wk.qblk, 0, p), tile_range(wk.qblk, 1, p)};
-    const int lo = r[0].lo;
-    const int hi = r[1].active ? r[1].hi : r[0].hi;
-    ok = warp_wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
-    q_phase[0] ^= 1u;
-    if (ok && r[1].active) {
+    const WorkItem wk = decode_work<kRanges>(w, p);
+    const TileRange r[2] = {tile_range<kRanges>(wk, 0, p), tile_range<kRanges>(wk, 1, p)};
+    const bool live0 = live<kRanges>(r[0]), live1 = live<kRanges>(r[1]);
+    int lo, hi;
+    if constexpr (kRanges) {
+      if (!live0 && !live1) continue;
+      lo = !live1 ? r[0].lo : (!live0 ? r[1].lo : min(r[0].lo, r[1].lo));
+      hi = !live1 ? r[0].hi : (!live0 ? r[1].hi : max(r[0].hi, r[1].hi));
+    } else {
+      lo = r[0].lo;
+      hi = r[1].active ? r[1].hi : r[0].hi;
+    }
+    if (live0) {
+      ok = warp_wait_phase(&ctl->q_full[0], q_phase[0], ctl, p, kSiteMmaQFull, true);
+      q_phase[0] ^= 1u;
+    }
+    if (ok && live1) {
       ok = warp_wait_phase(&ctl->q_full[1], q_phase[1], ctl, p, kSiteMmaQFull, true);
       q_phase[1] ^= 1u;
     }
@@ -488,7 +550,7 @@ __device__ __forceinline__ float max128(const float (&x)[128]) {
   return fmaxf(fmax3(c[0], c[1], c[2]), fmaxf(c[3], c[4]));
 }
 
-template <class C>
+template <class C, bool kRanges>
 __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t tmem, int warp, int lane) {
   const int quad = warp & 3;
   const int row_in_tile = quad * 32 + lane;
@@ -500,10 +562,22 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
   for (int i = 0;; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const WorkItem wk = decode_work(w, p);
-    const TileRange r = tile_range(wk.qblk, t, p);
+    const WorkItem wk = decode_work<kRanges>(w, p);
+    const TileRange r = tile_range<kRanges>(wk, t, p);
     if (!r.active) continue;
     const int qrow = r.q0 + row_in_tile;
+    if (kRanges && r.lo >= r.hi) {  // no row of this tile sees a key: O = 0, LSE = -inf
+      if (qrow < p.N) {
+        const size_t row_elem = ((static_cast<size_t>(wk.b) * p.N + qrow) * p.Hq + wk.h) * C::kDout;
+        constexpr int kVec = C::kDout * (C::kOut == kOutBf16 ? 2 : 4) / 16;
+        uint4* dst = C::kOut == kOutBf16 ? reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row_elem)
+                                         : reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.o) + row_elem);
+#pragma unroll 4
+        for (int i = 0; i < kVec; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+        p.lse[(static_cast<size_t>(wk.b) * p.Hq + wk.h) * p.N + qrow] = -CUDART_INF_F;
+      }
+      continue;
+    }
     float cs = p.scale_log2;
     float out_mult = 1.0f;
     if (C::kEsize == 1) {
@@ -511,8 +585,13 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
       out_mult = __ldg(p.v_scale + wk.hkv);
     }
     // Key columns this row may see: [key_lo, key_hi).
-    const int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;
-    const int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
+    int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;
+    int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
+    if (kRanges && qrow < p.N) {
+      const size_t ix = static_cast<size_t>(wk.b) * p.N + qrow;
+      key_lo = max(key_lo, __ldg(p.key_lo + ix));
+      key_hi = min(key_hi, __ldg(p.key_hi + ix));
+    }
 
     float m_used = -CUDART_INF_F;
     float l = 0.0f;
@@ -534,8 +613,11 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
         tmem_wait_ld();
       }
       const int kbase = j * 128;
-      const bool need_mask = (kbase + 128 > p.N) || (p.causal && kbase + 127 > r.q0) ||
-                             (p.window > 0 && kbase <= r.last_row - p.window);
+      // Mask when some row sees only part of the tile (with row ranges: some
+      // row of this warp).
+      const bool need_mask = kRanges ? __any_sync(0xFFFFFFFFu, kbase < key_lo || kbase + 128 > key_hi)
+                                     : (kbase + 128 > p.N) || (p.causal && kbase + 127 > r.q0) ||
+                                           (p.window > 0 && kbase <= r.last_row - p.window);
       if (need_mask) {
         const int vlo = key_lo - kbase;  // visible columns [vlo, vhi) of this tile
         const int vhi = key_hi - kbase;
@@ -680,8 +762,98 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
   }
 }
 
+// --------------------------------------------- per-tile K/V ranges (masks)
+// One block of 128 threads per (batch, 128-row query tile): thread r takes
+// row q0 + r's visible keys [max(key_lo, 0, window start), min(key_hi, N,
+// row + 1 when causal)) and the block reduces them to the span of K/V tiles
+// [lo / 128, ceil(hi / 128)) that covers every non-empty row; (0, 0) when
+// no row of the tile sees a key.
+__global__ void __launch_bounds__(128) row_range_tiles_kernel(const int* __restrict__ key_lo,
+                                                              const int* __restrict__ key_hi, int2* tile_kv,
+                                                              int N, int num_qtiles, int causal, int window) {
+  __shared__ int s_lo[4], s_hi[4];
+  const int b = blockIdx.x / num_qtiles;
+  const int qt = blockIdx.x - b * num_qtiles;
+  const int row = qt * 128 + static_cast<int>(threadIdx.x);
+  int lo = INT_MAX, hi = INT_MIN;
+  if (row < N) {
+    const size_t ix = static_cast<size_t>(b) * N + row;
+    int a = max(0, __ldg(key_lo + ix));
+    int e = min(N, __ldg(key_hi + ix));
+    if (window > 0) a = max(a, row - window + 1);
+    if (causal) e = min(e, row + 1);
+    if (a < e) {
+      lo = a;
+      hi = e;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_lo[threadIdx.x >> 5] = lo;
+    s_hi[threadIdx.x >> 5] = hi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    lo = min(min(s_lo[0], s_lo[1]), min(s_lo[2], s_lo[3]));
+    hi = max(max(s_hi[0], s_hi[1]), max(s_hi[2], s_hi[3]));
+    tile_kv[blockIdx.x] = lo < hi ? make_int2(lo / 128, (hi + 127) / 128) : make_int2(0, 0);
+  }
+}
+
+// With per-row key ranges the cost of a work item depends on the data, so
+// the (batch, query block) pairs are ranked by the number of K/V tiles their
+// two query tiles visit, most first, before the launch: the kernel's
+// boustrophedon deal over a descending ranking then gives every CTA about
+// the same work.  One block, a bitonic sort of (cost, index) keys in shared
+// memory (kOrderMaxPairs at most; beyond that the host passes no order and
+// the default ranking is used).  Ties keep index order, so the ranking and
+// the results do not vary from run to run.
+constexpr int kOrderMaxPairs = 16384;
+
+__global__ void __launch_bounds__(1024) order_items_kernel(const int2* __restrict__ tile_kv, int* order, int n,
+                                                           int num_qblk, int num_qtiles, int pow2) {
+  extern __shared__ unsigned long long keys[];
+  for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
+    unsigned long long key = ~0ull;  // padding sorts last
+    if (i < n) {
+      const int b = i / num_qblk;
+      const int qb = i - b * num_qblk;
+      const int2 t0 = tile_kv[static_cast<size_t>(b) * num_qtiles + 2 * qb];
+      int cost = max(0, t0.y - t0.x);
+      if (2 * qb + 1 < num_qtiles) {
+        const int2 t1 = tile_kv[static_cast<size_t>(b) * num_qtiles + 2 * qb + 1];
+        cost += max(0, t1.y - t1.x);
+      }
+      key = (static_cast<unsigned long long>(0x7FFFFFFF - cost) << 32) | static_cast<unsigned>(i);
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= pow2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], c = keys[ixj];
+          const bool ascending = (i & k) == 0;
+          if (ascending ? (a > c) : (a < c)) {
+            keys[i] = c;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) order[i] = static_cast<int>(keys[i] & 0xFFFFFFFFull);
+}
+
 // ------------------------------------------------------------- the kernel
-template <class C>
+template <class C, bool kRanges>
 __global__ void __launch_bounds__(C::kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -725,14 +897,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 
   if (warp < 8) {
     regs_increase<C::kSoftmaxRegs>();
-    softmax_role<C>(warp >> 2, p, ctl, tmem, warp, lane);
+    softmax_role<C, kRanges>(warp >> 2, p, ctl, tmem, warp, lane);
   } else {
     regs_decrease<C::kControlRegs>();
     if (warp == 8) {
-      mma_role<C>(p, ctl, smem, tmem);
+      mma_role<C, kRanges>(p, ctl, smem, tmem);
       __syncwarp();
     } else if (warp == 9) {
-      if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, ctl, smem);
+      if (lane == 0) producer_role<C, kRanges>(&tm_q, &tm_k, &tm_v, p, ctl, smem);
       __syncwarp();
     }
   }

@@ -119,28 +119,37 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize
   return r == CUDA_SUCCESS ? EA_OK : EA_EINVAL;
 }
 
-template <class C>
-int launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const ea::FwdParams& p,
-                     const DeviceState& ds, cudaStream_t stream) {
+template <class C, bool kRanges>
+int launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const ea::FwdParams& p,
+                   const DeviceState& ds, cudaStream_t stream) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(ea::attn_fwd_sm100<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(ea::attn_fwd_sm100<C, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
       return EA_ELAUNCH;
     // The warpgroups re-split the registers the block is launched with
     // (setmaxnreg); a block launched with fewer than the split assumes would
     // wait in setmaxnreg forever, so refuse to launch it.
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, ea::attn_fwd_sm100<C>) != cudaSuccess || fa.numRegs < C::kLaunchRegs)
+    if (cudaFuncGetAttributes(&fa, ea::attn_fwd_sm100<C, kRanges>) != cudaSuccess || fa.numRegs < C::kLaunchRegs)
       return EA_ELAUNCH;
     attr_done[dev] = true;
   }
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
-  ea::attn_fwd_sm100<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  ea::attn_fwd_sm100<C, kRanges><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
+}
+
+// The kernel variant with per-row key ranges is a separate instantiation,
+// so the plain causal / window kernel carries none of its code.
+template <class C>
+int launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const ea::FwdParams& p,
+                     const DeviceState& ds, cudaStream_t stream) {
+  return p.tile_kv != nullptr ? launch_variant<C, true>(tq, tk, tv, p, ds, stream)
+                              : launch_variant<C, false>(tq, tk, tv, p, ds, stream);
 }
 
 // fp32 -> (hi, lo) bf16 split.  x = hi + lo + O(2^-17 |x|); the attention
@@ -205,13 +214,17 @@ int launch_split(SplitJob q, SplitJob k, SplitJob v, int num_sms, cudaStream_t s
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-}  // namespace
+int forward_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, int causal, int window, const int* key_lo, const int* key_hi, const int2* tile_kv,
+                   const int* item_order, int num_qtiles, float scale, int dtype, const float* q_scale,
+                   const float* k_scale, const float* v_scale, DeviceState* ds, cudaStream_t stream);
 
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
-             int causal, int window, float scale, int dtype, const float* q_scale, const float* k_scale,
-             const float* v_scale, void* stream_ptr) {
+// The forward behind attn_fwd (key_lo == key_hi == null) and attn_fwd_masked:
+// argument checks, the per-tile range pre-pass when row ranges are given,
+// then forward_launch.
+int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                 int d, int causal, int window, const int* key_lo, const int* key_hi, float scale, int dtype,
+                 const float* q_scale, const float* k_scale, const float* v_scale, void* stream_ptr) {
   // ---- arguments that need no device
   if (!q || !k || !v || !o || !lse) return EA_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return EA_EINVAL;
@@ -249,9 +262,74 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return EA_EINVAL;
   if (fp8 && (check_range(q_scale, Hq * 4) || check_range(k_scale, Hkv * 4) || check_range(v_scale, Hkv * 4)))
     return EA_EINVAL;
+  const bool ranges = key_lo != nullptr;
+  const long long num_qtiles = (N + 127) / 128;
+  if (ranges && (check_range(key_lo, static_cast<size_t>(B) * N * 4) ||
+                 check_range(key_hi, static_cast<size_t>(B) * N * 4)))
+    return EA_EINVAL;
 
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
+  // Per-row key ranges: reduce them to a K/V tile range per 128-row query
+  // tile, then rank the (batch, query block) pairs by cost (stream-ordered
+  // scratch from the pool, freed after the launch).
+  int2* tile_kv = nullptr;
+  int* order = nullptr;
+  if (ranges) {
+    const long long pairs = static_cast<long long>(B) * num_qblk;
+    const size_t tb = static_cast<size_t>(B) * num_qtiles * sizeof(int2);
+    const size_t ob = static_cast<size_t>(pairs) * sizeof(int);
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, tb + ob, ds->pool, stream) != cudaSuccess) return EA_ENOMEM;
+    tile_kv = static_cast<int2*>(scratch);
+    ea::row_range_tiles_kernel<<<static_cast<unsigned>(B * num_qtiles), 128, 0, stream>>>(
+        key_lo, key_hi, tile_kv, N, static_cast<int>(num_qtiles), causal, window > 0 ? window : 0);
+    rc = cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
+    if (rc == EA_OK && pairs <= ea::kOrderMaxPairs && g_order == 2) {
+      int pow2 = 1;
+      while (pow2 < pairs) pow2 <<= 1;
+      const size_t smem = static_cast<size_t>(pow2) * sizeof(unsigned long long);
+      static bool attr_done[kMaxDevices] = {};
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(ea::order_items_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 ea::kOrderMaxPairs * static_cast<int>(sizeof(unsigned long long))) != cudaSuccess)
+          rc = EA_ELAUNCH;
+        else
+          attr_done[dev] = true;
+      }
+      if (rc == EA_OK) {
+        order = reinterpret_cast<int*>(static_cast<char*>(scratch) + tb);
+        ea::order_items_kernel<<<1, 1024, smem, stream>>>(tile_kv, order, static_cast<int>(pairs),
+                                                          static_cast<int>(num_qblk), static_cast<int>(num_qtiles),
+                                                          pow2);
+        if (cudaGetLastError() != cudaSuccess) rc = EA_ELAUNCH;
+      }
+    }
+    if (rc != EA_OK) {
+      cudaFreeAsync(scratch, stream);
+      return rc;
+    }
+  }
+  rc = forward_launch(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, key_lo, key_hi, tile_kv, order,
+                      static_cast<int>(num_qtiles), scale, dtype, q_scale, k_scale, v_scale, ds, stream);
+  if (tile_kv) cudaFreeAsync(tile_kv, stream);
+  return rc;
+}
+
+int forward_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, int causal, int window, const int* key_lo, const int* key_hi, const int2* tile_kv,
+                   const int* item_order, int num_qtiles, float scale, int dtype, const float* q_scale,
+                   const float* k_scale, const float* v_scale, DeviceState* ds, cudaStream_t stream) {
+  const bool fp8 = dtype == EA_FP8_E4M3;
+  const long long num_qblk = (N + 255) / 256;
+  int rc = EA_OK;
   ea::FwdParams p{};
+  p.key_lo = key_lo;
+  p.key_hi = key_hi;
+  p.tile_kv = tile_kv;
+  p.item_order = item_order;
+  p.num_qtiles = num_qtiles;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
@@ -268,7 +346,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_qblk = static_cast<int>(num_qblk);
   p.num_work = static_cast<int>(B * Hq * num_qblk);
-  p.order = g_order;
+  p.order = g_order == 1 ? 1 : 0;
   p.skip_first_kv = g_skip_arrive_once;
   p.timeout_ns = g_timeout_ns;
   g_skip_arrive_once = 0;
@@ -316,6 +394,26 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   return rc;
 }
 
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+             int causal, int window, float scale, int dtype, const float* q_scale, const float* k_scale,
+             const float* v_scale, void* stream) {
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, nullptr, nullptr, scale, dtype, q_scale,
+                      k_scale, v_scale, stream);
+}
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                    int d, int causal, int window, const int32_t* key_lo, const int32_t* key_hi, float scale,
+                    int dtype, const float* q_scale, const float* k_scale, const float* v_scale, void* stream) {
+  if (!key_lo || !key_hi) return EA_EINVAL;
+  if (!aligned(key_lo, 4) || !aligned(key_hi, 4)) return EA_EALIGN;
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, key_lo, key_hi, scale, dtype, q_scale,
+                      k_scale, v_scale, stream);
+}
+
 int attn_get_last_error(void* stream_ptr, int* device_code, int* site) {
   if (device_code) *device_code = 0;
   if (site) *site = 0;
@@ -357,7 +455,7 @@ int attn_set_option(int option, long long value) {
       g_max_ctas = static_cast<int>(value);
       return EA_OK;
     case EA_OPT_SCHEDULE_ORDER:
-      if (value != 0 && value != 1) return EA_EINVAL;
+      if (value < 0 || value > 2) return EA_EINVAL;
       g_order = static_cast<int>(value);
       return EA_OK;
     case EA_OPT_SKIP_ARRIVE_ONCE:
@@ -489,7 +587,7 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_qblk = static_cast<int>(num_qblk);
   p.num_work = static_cast<int>(B * Hq * num_qblk);
-  p.order = g_order;
+  p.order = g_order == 1 ? 1 : 0;
   p.skip_first_kv = 0;
   p.timeout_ns = g_timeout_ns;
 

@@ -208,6 +208,8 @@ def shard_inputs(inp: Dict[str, Optional[torch.Tensor]], q_lo: int, q_hi: int, k
         out[name] = inp[name][:, :, lo:hi, :].contiguous()
         s = inp[name + "_scale"]
         out[name + "_scale"] = None if s is None else s[lo:hi].contiguous()
+    # per-row key ranges are shared by all heads: every shard keeps them whole
+    out["key_lo"], out["key_hi"] = inp.get("key_lo"), inp.get("key_hi")
     return out
 
 

@@ -101,6 +101,40 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              void* stream);
 
 /*
+ * attn_fwd_masked -- attn_fwd with a per-row key range on top of the
+ * causal and window masks.
+ *
+ * What it computes: the same O and LSE, where the mask -- what decides which
+ * queries see which keys (Hacker News discussion, item 40939398) -- also
+ * holds one contiguous range of visible keys per query row, the simplest
+ * form of the richer masks of the FlashMask work that "FlashAttention-2
+ * (PL)" lists in its literature section.  Query row i of batch b sees key j
+ * iff key_lo[b*N + i] <= j < key_hi[b*N + i] and the causal / window
+ * conditions of attn_fwd hold.  Examples: packed documents (key_lo = the
+ * row's document start, key_hi = its end, causal = 1), a prefix-LM mask
+ * (key_lo = 0, key_hi = max(prefix, i + 1), causal = 0), a sliding window
+ * that varies by row.
+ *
+ *   key_lo, key_hi  device int32 arrays [B, N] (row-major), 4-byte aligned,
+ *                   owned by the caller, shared by all heads; any values
+ *                   (ranges are clipped to [0, N); lo >= hi: no key).
+ *   all other arguments as attn_fwd.
+ *
+ * A row that sees no key gets O = 0 and LSE = -inf.  The cost follows the
+ * visible keys: each 128-row query tile visits only the K/V tiles spanned by
+ * its rows' ranges (a small kernel reduces the ranges per tile first, into
+ * stream-ordered scratch from the library's pool that goes back to the pool
+ * after the launch).
+ *
+ * Errors: those of attn_fwd, plus EA_EINVAL for a NULL key_lo / key_hi or
+ * arrays that are not device allocations of B*N int32, EA_EALIGN for
+ * misaligned ones, EA_ENOMEM when the pool cannot supply the tile table.
+ */
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                    int d, int causal, int window, const int32_t* key_lo, const int32_t* key_hi, float scale,
+                    int dtype, const float* q_scale, const float* k_scale, const float* v_scale, void* stream);
+
+/*
  * attn_get_last_error -- synchronise `stream`, then read and clear the
  * current device's error word.  *device_code receives 0 or the recorded
  * failure kind (1 = wait timed out), *site the pipeline wait that failed
@@ -118,7 +152,11 @@ const char* attn_status_string(int status);
  *                           (default 2e9 ns).
  *   EA_OPT_MAX_CTAS         cap on persistent CTAs per launch (0 = one per SM).
  *   EA_OPT_SCHEDULE_ORDER   0 = heaviest query blocks first (default),
- *                           1 = lightest first.  Results do not depend on it.
+ *                           1 = lightest first, 2 = with per-row key ranges,
+ *                           (batch, query block) pairs ranked by the K/V
+ *                           tiles they visit, most first (better balance
+ *                           across SMs, less reuse of K/V in L2; otherwise
+ *                           as 0).  Results do not depend on it.
  *   EA_OPT_SKIP_ARRIVE_ONCE test hook: the next launch's load warp skips its
  *                           first key/value copy, so the consumer's bounded
  *                           wait runs out and reports EA_EDEVICE_TIMEOUT.

@@ -175,3 +175,31 @@ def test_reference_arm_on_a_decode_workload():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["config"]["Nq"] == 2 and j["config"]["Nk"] == 8192
     assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_on_the_document_mask_workload():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+           "bf16_doccausal_b2h16_n16384_d128", "--steps", "3", "--warmup", "3", "--ref-seconds", "3"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr
+    lines = [l for l in proc.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["config"]["row_ranges"].startswith("documents")
+    assert j["value"] > 0
+
+
+def test_pairs_for_rows_with_ranges_brute_force():
+    from exact_io_aware_78_b200.inputs import make_row_ranges
+    N = 60
+    lo, hi = make_row_ranges("random", 1, N, 8)
+    lo, hi = lo[0].numpy(), hi[0].numpy()
+    rows = [0, 3, 17, 59, 30]
+    for causal in (False, True):
+        for window in (0, 5):
+            want = 0
+            for i in rows:
+                for j in range(N):
+                    if lo[i] <= j < hi[i] and (not causal or j <= i) and (window <= 0 or j > i - window):
+                        want += 1
+            assert bench.pairs_for_rows(rows, N, causal, window, lo, hi) == want

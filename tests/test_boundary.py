@@ -27,7 +27,7 @@ def lib(lib_path):
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_get_last_error", "attn_status_string", "attn_set_option", "attn_shutdown",
-         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode"])
+         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked"])
 
 
 def test_library_exports_every_declared_symbol(lib_path):
@@ -48,7 +48,8 @@ def test_version_and_status_strings(lib):
 
 def test_options_validation(lib):
     assert lib.attn_set_option(B.EA_OPT_WAIT_TIMEOUT_NS, 10) == B.EA_EINVAL
-    assert lib.attn_set_option(B.EA_OPT_SCHEDULE_ORDER, 2) == B.EA_EINVAL
+    assert lib.attn_set_option(B.EA_OPT_SCHEDULE_ORDER, 3) == B.EA_EINVAL
+    assert lib.attn_set_option(B.EA_OPT_SCHEDULE_ORDER, -1) == B.EA_EINVAL
     assert lib.attn_set_option(B.EA_OPT_MAX_CTAS, -1) == B.EA_EINVAL
     assert lib.attn_set_option(99, 0) == B.EA_EINVAL
     assert lib.attn_set_option(B.EA_OPT_SCHEDULE_ORDER, 0) == B.EA_OK
@@ -101,6 +102,33 @@ def test_argument_errors(lib, kw, code):
         assert rc == code
 
 
+def call_masked(lib, lo=P, hi=P, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B_=1, Hq=2, Hkv=1, N=128, d=128, causal=1, window=0, scale=0.125,
+             dtype=B.EA_BF16, qs=None, ks=None, vs=None)
+    a.update(kw)
+    return lib.attn_fwd_masked(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B_"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                               a["causal"], a["window"], lo, hi, a["scale"], a["dtype"], a["qs"], a["ks"], a["vs"],
+                               None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lo=None), B.EA_EINVAL),
+    (dict(hi=None), B.EA_EINVAL),
+    (dict(lo=P + 2), B.EA_EALIGN),
+    (dict(hi=P + 1), B.EA_EALIGN),
+    (dict(q=None), B.EA_EINVAL),                  # the checks of attn_fwd apply too
+    (dict(causal=2), B.EA_EINVAL),
+    (dict(d=96), B.EA_EUNSUPPORTED),
+    (dict(), None),                                # valid: reaches the device step
+])
+def test_masked_argument_errors(lib, kw, code):
+    rc = call_masked(lib, **kw)
+    if code is None:
+        assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
+    else:
+        assert rc == code
+
+
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     import torch
     if torch.cuda.is_available():
@@ -113,6 +141,9 @@ def test_python_binding_rejects_bad_layouts():
     q = torch.zeros(1, 8, 2, 64)
     with pytest.raises(ValueError):
         B.attn_fwd(q, q, q, q, torch.zeros(1, 2, 8))          # CPU tensors
+    r = torch.zeros(1, 8, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        B.attn_fwd_masked(q, q, q, q, torch.zeros(1, 2, 8), r, r)
 
 
 def call_decode(lib, q=P, k=P, v=P, o=P, lse=P, B_=1, Hq=8, Hkv=2, Nq=1, Nk=4096, d=128, causal=1, window=0,

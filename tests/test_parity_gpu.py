@@ -9,7 +9,7 @@ from exact_io_aware_78_b200 import _binding as Bn
 from exact_io_aware_78_b200.inputs import WORKLOADS, make_inputs, sample_rows, workload_inputs
 from oracle import attention_ref
 
-from gpu_helpers import assert_close, case, oracle_view, run_gpu
+from gpu_helpers import assert_close, case, oracle_view, ranges_view, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -82,7 +82,8 @@ def test_workload_sampled_rows(name):
     # properties that hold at any size
     assert np.isfinite(O).all() and np.isfinite(L).all()
     q, k, v = oracle_view(inp, w.dtype)
-    Oref, Lref = attention_ref(q, k, v, w.causal, w.window, w.scale, rows=rows)
+    lo, hi = ranges_view(inp)
+    Oref, Lref = attention_ref(q, k, v, w.causal, w.window, w.scale, rows=rows, key_lo=lo, key_hi=hi)
     if rows is not None:
         O, L = O[:, rows], L[:, :, rows]
     assert_close(O, L, Oref, Lref, w.dtype, name)
