@@ -7,6 +7,10 @@ TMA loads, S = Q K^T, online softmax, O += P V, epilogue) over one batch of
 the workload's seeded synthetic inputs, already resident in HBM.  Each step
 is timed with CUDA events on the launching stream; between steps a 256 MiB
 buffer is written to flush the 126 MB L2 (not timed).  Prints one JSON line.
+Other workloads: decode_* time one attn_fwd_decode call per step (key-range
+and combine kernels); bf16_doccausal_* one attn_fwd_masked call (tile-range
+pre-pass and the range variant of the forward kernel); bwd_* one attn_bwd
+call (stats pass, dK/dV kernel, dQ kernel) after an untimed forward.
 
 Multi-GPU (torchrun): one process per GPU, each runs its own replica of the
 workload (independent problems, no collective on the data path); the
@@ -30,8 +34,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_78_b200 import accounting  # noqa: E402
-from exact_io_aware_78_b200.inputs import (DECODE_WORKLOADS, DEFAULT_BENCH_WORKLOAD, WORKLOADS,  # noqa: E402
-                                           decode_workload_inputs, head_shard, shard_inputs, workload_inputs)
+from exact_io_aware_78_b200.inputs import (BWD_WORKLOADS, DECODE_WORKLOADS, DEFAULT_BENCH_WORKLOAD,  # noqa: E402
+                                           WORKLOADS, decode_workload_inputs, head_shard, make_grad_output,
+                                           shard_inputs, workload_inputs)
 
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -42,7 +47,10 @@ KERNEL_SOURCES = {
                 "exact_io_aware_78_b200/csrc/exactattn.cu"],
     "decode": ["exact_io_aware_78_b200/csrc/decode_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_api.cuh",
                "exact_io_aware_78_b200/csrc/sm100_ptx.cuh"],
+    "backward": ["exact_io_aware_78_b200/csrc/attn_bwd_kernel.cuh", "exact_io_aware_78_b200/csrc/backward_api.cuh",
+                 "exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh"],
 }
+METRIC_BWD = "attention bwd TFLOP/s (5 products of 2*d FLOPs per attended pair), 1 GPU"
 
 
 def kernel_source_hash(kind: str = "prefill") -> str:
@@ -70,7 +78,8 @@ def load_traffic(workload: str):
     with open(path) as f:
         data = json.load(f)
     ent = data.get(workload)
-    kind = "decode" if workload.startswith("decode_") else "prefill"
+    kind = ("decode" if workload.startswith("decode_") else "backward" if workload.startswith("bwd_")
+            else "prefill")
     if not ent or ent.get("kernel_source_hash") != kernel_source_hash(kind):
         return None
     return ent.get("dram_bytes_per_launch")
@@ -273,6 +282,44 @@ def is_decode(w) -> bool:
     return w.name in DECODE_WORKLOADS
 
 
+def is_backward(w) -> bool:
+    return w.name in BWD_WORKLOADS
+
+
+class BackwardOracleSampler:
+    """Times the float64 backward oracle one (b, h) query head at a time
+    (with its key/value head), continuing where it stopped."""
+
+    def __init__(self, w):
+        inp = workload_inputs(w)
+        self.w = w
+        self.qkv = [inp[n].to(torch.float64).numpy() for n in "qkv"]
+        self.do = make_grad_output(w.B, w.N, w.Hq, w.d, w.seed + 3).to(torch.float64).numpy()
+        self.cursor = 0
+
+    def run(self, budget_s: float):
+        """Returns (seconds, backward FLOPs covered, query rows done)."""
+        from oracle import attention_bwd_ref  # CPU baseline leg only
+
+        w = self.w
+        q, k, v = self.qkv
+        pairs = accounting.attended_pairs(w.N, w.causal, w.window)
+        flops = 0.0
+        rows_done = 0
+        t0 = time.perf_counter()
+        while True:
+            b, h = divmod(self.cursor % (w.B * w.Hq), w.Hq)
+            self.cursor += 1
+            kh = h // w.group
+            attention_bwd_ref(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, kh:kh + 1], v[b:b + 1, :, kh:kh + 1],
+                              self.do[b:b + 1, :, h:h + 1], w.causal, w.window, w.scale)
+            flops += 10.0 * w.d * pairs
+            rows_done += w.N
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        return time.perf_counter() - t0, flops, rows_done
+
+
 def run_reference(args, w, world, rank):
     if rank != 0:
         return
@@ -280,7 +327,8 @@ def run_reference(args, w, world, rank):
     flops_done = 0.0
     rows_total = 0
     per_step_budget = min(20.0, args.ref_seconds / max(1, args.steps + args.warmup))
-    sampler = DecodeOracleSampler(w) if is_decode(w) else OracleSampler(w)
+    sampler = (DecodeOracleSampler(w) if is_decode(w) else BackwardOracleSampler(w) if is_backward(w)
+               else OracleSampler(w))
     for i in range(args.warmup + args.steps):
         dt, fl, rows = sampler.run(per_step_budget)
         if i >= args.warmup:
@@ -289,12 +337,13 @@ def run_reference(args, w, world, rank):
             rows_total += rows
     value = flops_done / sum(times) / 1e12
     unit_desc = ("query rows (all Nq rows of consecutive (b,h) heads)" if is_decode(w) else
+                 "query rows (all N rows of consecutive (b,h) heads, backward)" if is_backward(w) else
                  "query rows (128-row chunks of consecutive (b,h) heads)")
     sample = (f"{rows_total} {unit_desc} of {w.name} over "
               f"{args.steps} steps of ~{per_step_budget:.3g} s, numpy float64 two-pass oracle; "
               f"TFLOP/s counts attended-pair FLOPs")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC_BWD if is_backward(w) else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
@@ -467,6 +516,134 @@ def run_cuda(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_backward_cuda(args, w, world, rank, local):
+    """One backward step (attn_bwd: the stats pass, the dK/dV kernel and the
+    dQ kernel) per timed iteration; O and LSE come from one untimed forward."""
+    import exact_io_aware_78_b200 as ea
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    w_job = w
+    inp = workload_inputs(w)
+    inp["do"] = make_grad_output(w.B, w.N, w.Hq, w.d, w.seed + 3)
+    if args.shard == "heads":
+        w, q_lo, q_hi, kv_lo, kv_hi = head_shard(w_job, world, rank)
+        do_full = inp["do"]
+        inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
+        inp["do"] = do_full[:, :, q_lo:q_hi].contiguous()
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = ea.forward(q, k, v, causal=w.causal, window=w.window, scale=w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, w.causal, w.window, w.scale, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st, code, site = ea.attn_get_last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {code} at site {site} during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    st, code, site = ea.attn_get_last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {code} at site {site} in the timed region")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = dist_max(sum(step_ms), world, dev)
+    flops = accounting.bwd_flops(w)
+    if args.shard == "heads":
+        value = sharded_tflops(accounting.bwd_flops(w_job), args.steps, total_ms)
+    else:
+        value = job_tflops(flops, args.steps, world, total_ms)
+
+    # e2e: the public call with the step's inputs copied from pinned host memory
+    host_in = [(t, t.cpu().pin_memory()) for t in (q, k, v, o, lse, do)]
+    host_out = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in (dq, dk, dv)]
+    e2e_steps = max(3, min(args.steps, 50))
+    es = torch.cuda.Event(enable_timing=True)
+    ee = torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(e2e_steps + 2):
+        flush.zero_()
+        es.record(stream)
+        for dst, src in host_in:
+            dst.copy_(src, non_blocking=True)
+        step()
+        for src, dst in host_out:
+            dst.copy_(src, non_blocking=True)
+        ee.record(stream)
+        ee.synchronize()
+        if i >= 2:
+            e2e_ms.append(es.elapsed_time(ee))
+    e2e_total = dist_max(sum(e2e_ms), world, dev)
+    if args.shard == "heads":
+        e2e_value = sharded_tflops(accounting.bwd_flops(w_job), e2e_steps, e2e_total)
+    else:
+        e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
+    h2d = sum(src.numel() * src.element_size() for _, src in host_in)
+    d2h = sum(dst.numel() * dst.element_size() for _, dst in host_out)
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    launch_ms = statistics.mean(step_ms)
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC_BWD,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "strong" if args.shard == "heads" else "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**workload_config(w_job), "pass": "backward", "flops_per_step": accounting.bwd_flops(w_job),
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "parallelism": (f"head shards x{world}" if args.shard == "heads" else
+                                   f"replicas x{world}" if world > 1 else "single GPU")},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": load_traffic(w.name),
+                     "peak_source": f"{peak_kind} bf16 burst (kernel timed alone)",
+                     "peak_sustained": peaks["bf16_tflops_sustained"],
+                     "frac_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     "algorithmic_bytes": accounting.bwd_bytes(w),
+                     "kernel_source_hash": kernel_source_hash("backward"),
+                     "note": "achieved over the whole step (stats pass + dK/dV kernel + dQ kernel)"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 3,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        dt, fl, rows = BackwardOracleSampler(w).run(args.cpu_seconds)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"{rows} query rows (all rows of consecutive (b,h) heads) of {w.name} "
+                                          f"in {dt:.1f} s, numpy float64 backward oracle; TFLOP/s counts 10*d "
+                                          f"FLOPs per attended pair"}
+    print(json.dumps(line), flush=True)
+
+
 def run_decode_cuda(args, w, world, rank, local):
     """A decode step (attn_fwd_decode): Nq new query rows per (b, h) against a
     cache of Nk keys.  HBM-bound, so the roofline is the measured copy
@@ -594,7 +771,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD,
-                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(BWD_WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="with several GPUs: each runs its own replica of the workload (weak scaling), or the "
@@ -607,14 +784,15 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = WORKLOADS[args.workload] if args.workload in WORKLOADS else DECODE_WORKLOADS[args.workload]
+    w = {**WORKLOADS, **DECODE_WORKLOADS, **BWD_WORKLOADS}[args.workload]
     if args.impl == "reference":
         # host-only: rank 0 times the oracle, other ranks exit without work
         run_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
     world, rank, local = init_dist()
     try:
-        (run_decode_cuda if is_decode(w) else run_cuda)(args, w, world, rank, local)
+        (run_decode_cuda if is_decode(w) else run_backward_cuda if is_backward(w) else run_cuda)(
+            args, w, world, rank, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -32,6 +32,8 @@ _SIGNATURES = {
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_void_p]),
+    "attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7 + [ctypes.c_float, ctypes.c_int,
+                                                                                ctypes.c_void_p]),
     "attn_get_last_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -178,6 +180,49 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
     _forward_call(q, k, v, o, lse, causal, window, key_lo, key_hi, scale, q_scale, k_scale, v_scale, stream)
     return o, lse
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, causal: bool = False,
+             window: int = 0, scale: Optional[float] = None, stream=None) -> None:
+    """Queue dQ, dK, dV = the backward of attn_fwd (bf16) on `stream`.
+    q, o, dout, dq [B,N,Hq,d]; k, v, dk, dv [B,N,Hkv,d]; lse [B,Hq,N] fp32;
+    all contiguous CUDA tensors on one device; o and lse from the forward."""
+    lib = load_library()
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, N, H, d]")
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    want = {"q": (q, (B, N, Hq, d)), "k": (k, (B, N, Hkv, d)), "v": (v, (B, N, Hkv, d)), "o": (o, (B, N, Hq, d)),
+            "dout": (dout, (B, N, Hq, d)), "dq": (dq, (B, N, Hq, d)), "dk": (dk, (B, N, Hkv, d)),
+            "dv": (dv, (B, N, Hkv, d))}
+    for name, (t, shape) in want.items():
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor of shape {shape}")
+    if not lse.is_cuda or lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 CUDA tensor [B, Hq, N]")
+    if len({t.device for t in (q, k, v, o, lse, dout, dq, dk, dv)}) != 1:
+        raise ValueError("all tensors must be on one device")
+    if scale is None:
+        scale = d ** -0.5
+    device = q.device
+    with torch.cuda.device(device):
+        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, d, int(bool(causal)),
+                          int(window), float(scale), EA_BF16, _stream_handle(stream, device))
+    if st != EA_OK:
+        raise AttnError(st, "attn_bwd")
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, causal: bool = False, window: int = 0, scale: Optional[float] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Allocate dQ, dK, dV on q's device and run attn_bwd; returns them."""
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, window, scale, stream)
+    return dq, dk, dv
 
 
 def attn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,

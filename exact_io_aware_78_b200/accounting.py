@@ -86,6 +86,22 @@ def algorithmic_bytes(w: Workload) -> int:
     return q + kv + o + lse + scales
 
 
+def bwd_flops(w: Workload) -> float:
+    """Backward FLOPs: five products of 2*d FLOPs per attended pair (S, dP,
+    dV, dK, dQ), 2.5 x the forward's; the recomputation of S and dP in a
+    second kernel is not counted."""
+    return 2.5 * flops(w)
+
+
+def bwd_bytes(w: Workload) -> int:
+    """Algorithmic bytes of a backward step: Q, K, V, O, dO (bf16) and LSE
+    read once; dQ, dK, dV written once."""
+    q = w.B * w.N * w.Hq * w.d * 2
+    kv = w.B * w.N * w.Hkv * w.d * 2
+    lse = w.B * w.Hq * w.N * 4
+    return 3 * q + 2 * kv + lse + q + 2 * kv
+
+
 def decode_pairs(Nq: int, Nk: int, causal: bool, window: int) -> int:
     """Attended (query, key) pairs of one (b, h) in a decode step: query i
     sits at position Nk - Nq + i."""

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "attn_fwd_kernel.cuh"
+#include "attn_bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "exactattn.h"
 
@@ -602,3 +603,5 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
     return EA_EINVAL;
   return launch_attention<ea::KernelCfg<2, 192, 128, ea::kOutF32Split>>(tq, tk, tv, p, ds, stream);
 }
+
+#include "backward_api.cuh"  // attn_bwd

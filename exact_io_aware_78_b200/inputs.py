@@ -70,6 +70,17 @@ WORKLOADS: Dict[str, Workload] = {
 # The workload the benchmark times by default (causal, B=4, H=16, N=2048, d=128).
 DEFAULT_BENCH_WORKLOAD = "bf16_causal_b4h16_n2048_d128"
 
+# Backward-pass workloads: the forward's inputs plus dO = make_grad_output(seed + 3).
+BWD_WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("bwd_bf16_causal_b4h16_n2048_d128", 4, 16, 16, 2048, 128, True, 0, "bf16", 2048,
+                 description="backward of causal self-attention"),
+        Workload("bwd_bf16_gqa_causal_b2h32kv8_n4096_d128", 2, 32, 8, 4096, 128, True, 0, "bf16", 4096,
+                 description="backward of grouped-query causal attention"),
+    ]
+}
+
 
 def _randn(seed: int, shape, mult: float = 1.0) -> torch.Tensor:
     g = torch.Generator(device="cpu")
@@ -122,6 +133,12 @@ def workload_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
     if w.mask:
         out["key_lo"], out["key_hi"] = make_row_ranges(w.mask, w.B, w.N, w.seed + 3, w.mask_min, w.mask_max)
     return out
+
+
+def make_grad_output(B: int, N: int, Hq: int, d: int, seed: int) -> torch.Tensor:
+    """dO = dL/dO for backward runs: N(0, 1) drawn on the CPU, stored bf16
+    [B, N, Hq, d]."""
+    return _randn(seed, (B, N, Hq, d)).to(torch.bfloat16)
 
 
 def make_row_ranges(kind: str, B: int, N: int, seed: int, min_len: int = 1, max_len: int = 0):

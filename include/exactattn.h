@@ -135,6 +135,48 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
                     int dtype, const float* q_scale, const float* k_scale, const float* v_scale, void* stream);
 
 /*
+ * attn_bwd -- queue the backward pass of attn_fwd (bf16) on `stream`: the
+ * gradients dQ, dK, dV of a scalar loss whose gradient with respect to O is
+ * dO.
+ *
+ * What it computes: with P = softmax(scale Q K^T + mask) recomputed tile by
+ * tile from Q, K and the forward's LSE (the N x N probabilities are never
+ * stored: "Flash Attention" concept note (heepie.pages.dev), "Tiling" and
+ * "FLOP != speed"), the chain rule of the forward definition:
+ *     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO o O),  dS = P o (dP - D),
+ *     dQ = scale dS K,  dK = scale dS^T Q
+ * with the query heads of a group summed into their key/value head's dK, dV.
+ *
+ *   q, k, v   the forward's inputs, bf16, layouts as attn_fwd.
+ *   o, lse    the forward's outputs for the same q, k, v, causal, window and
+ *             scale: o bf16 [B, N, Hq, d], lse fp32 [B, Hq, N].
+ *   dout      dL/dO, bf16 [B, N, Hq, d].
+ *   dq        output bf16 [B, N, Hq, d];  dk, dv  outputs bf16 [B, N, Hkv, d].
+ *   B, Hq, Hkv, N, d, causal, window, scale   as attn_fwd; dtype must be
+ *             EA_BF16; d is 64 or 128.
+ *   stream    cudaStream_t (NULL = default stream); the call is asynchronous.
+ * All pointers are device pointers owned by the caller; q, k, v, o, dout, dq,
+ * dk, dv 16-byte aligned, lse 4-byte aligned.
+ *
+ * Memory: 8 bytes per query row and head of per-row statistics come
+ * stream-ordered from the library's pool and go back to it on the stream.
+ * Results are deterministic: every gradient element is accumulated by one
+ * CTA in a fixed order (no atomics).
+ *
+ * Errors (returned synchronously, nothing queued): EA_EINVAL for NULL
+ * pointers, non-positive sizes, Hq not a multiple of Hkv, causal not 0/1, a
+ * non-positive or non-finite scale, an unknown dtype, sizes past the limits
+ * of attn_fwd, or buffers that are not device allocations large enough;
+ * EA_EUNSUPPORTED for fp8/fp32 inputs or d other than 64/128; EA_EALIGN;
+ * EA_ENOMEM when the pool cannot supply the statistics; EA_ECUDA without a
+ * usable sm_100 device; EA_ELAUNCH if a launch fails.  A device-side wait
+ * that runs past its limit is reported by attn_get_last_error.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+             void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, int window, float scale, int dtype,
+             void* stream);
+
+/*
  * attn_get_last_error -- synchronise `stream`, then read and clear the
  * current device's error word.  *device_code receives 0 or the recorded
  * failure kind (1 = wait timed out), *site the pipeline wait that failed

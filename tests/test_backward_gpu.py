@@ -1,0 +1,128 @@
+"""Parity of the attention backward (attn_bwd, through the C ABI) with the
+float64 oracle attention_bwd_ref on seeded bf16 inputs: every element of
+dQ, dK, dV for small shapes (GQA groups, d = 64 and 128, causal and windowed
+masks, ragged N), both with the oracle's own O and LSE fed to the kernels
+(the backward alone) and end to end after the tcgen05 forward; sampled
+checks at a benchmark size; determinism; the invariants of the softmax
+Jacobian (dK sums to zero over the keys of a head)."""
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_78_b200 as ea
+from exact_io_aware_78_b200.inputs import make_grad_output, make_inputs
+from oracle import attention_bwd_ref, attention_ref
+
+pytestmark = pytest.mark.gpu
+
+# Bars, relative to the size of each reference gradient: max |err| <= 2e-2 *
+# max |ref| and mean |err| <= 1e-2 * mean |ref|.  The kernels round P and dS
+# to bf16 (relative step 2^-9) before the products that consume them and
+# store bf16 gradients, and accumulate in fp32, so each gradient element
+# carries errors of a few 2^-9 of the typical element size.
+TOL_MAX, TOL_MEAN = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(lib_path):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    if torch.cuda.get_device_capability(0)[0] != 10:
+        pytest.skip("needs an sm_100 GPU")
+    torch.cuda.set_device(0)
+    ea.load_library(lib_path)
+
+
+def inputs(B, Hq, Hkv, N, d, seed):
+    inp = make_inputs(B, Hq, Hkv, N, d, "bf16", seed)
+    inp["do"] = make_grad_output(B, N, Hq, d, seed + 3)
+    return inp
+
+
+def compare(got, ref, what):
+    out = []
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        g = g.double().cpu().numpy()
+        assert np.isfinite(g).all(), f"{what}: non-finite {name}"
+        err = np.abs(g - r)
+        mx, mean = err.max() / np.abs(r).max(), err.mean() / np.abs(r).mean()
+        out.append(f"{name} max {mx:.2e} mean {mean:.2e}")
+        assert mx <= TOL_MAX and mean <= TOL_MEAN, f"{what}: {name} relative max {mx:.3e}, mean {mean:.3e}"
+    print(what, "; ".join(out))
+
+
+def run_case(B, Hq, Hkv, N, d, causal, window, seed, end_to_end):
+    inp = inputs(B, Hq, Hkv, N, d, seed)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    scale = d ** -0.5
+    q64, k64, v64, do64 = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    o_ref, l_ref = attention_ref(q64, k64, v64, causal, window, scale)
+    if end_to_end:
+        o, lse = ea.forward(q, k, v, causal=causal, window=window, scale=scale)
+    else:
+        o = torch.from_numpy(o_ref).to(torch.bfloat16).to(dev)
+        lse = torch.from_numpy(l_ref).float().to(dev)
+    grads = ea.backward(q, k, v, o, lse, do, causal=causal, window=window, scale=scale)
+    st, code, site = ea.attn_get_last_error()
+    assert st == 0, f"device error code {code} at wait site {site}"
+    ref = attention_bwd_ref(q64, k64, v64, do64, causal, window, scale, o=o_ref, lse=l_ref)
+    compare(grads, ref, f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} c{int(causal)} w{window} e2e{int(end_to_end)}")
+    return grads
+
+
+CASES = [
+    # B, Hq, Hkv, N, d, causal, window
+    (1, 1, 1, 128, 128, False, 0),
+    (1, 2, 2, 128, 128, True, 0),
+    (1, 2, 1, 300, 128, True, 0),        # ragged, GQA 2:1
+    (2, 4, 1, 257, 64, True, 0),         # GQA 4:1, d = 64
+    (1, 2, 2, 520, 128, False, 0),
+    (1, 2, 2, 700, 128, True, 100),      # window
+    (1, 4, 2, 384, 64, False, 50),       # window without causal
+    (1, 1, 1, 17, 128, True, 0),         # one partial tile
+    (2, 8, 8, 1024, 128, True, 0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}h{}kv{}n{}d{}c{}w{}".format(*c))
+def test_backward_alone(case):
+    run_case(*case, seed=5000 + case[3] + case[4], end_to_end=False)
+
+
+@pytest.mark.parametrize("case", CASES[1::3], ids=lambda c: "B{}h{}kv{}n{}d{}c{}w{}".format(*c))
+def test_forward_then_backward(case):
+    run_case(*case, seed=6000 + case[3], end_to_end=True)
+
+
+def test_benchmark_shape_sampled():
+    """B4 H16 N2048 d128 causal (the backward benchmark's shape): full GPU run,
+    the oracle on four (b, h) heads, every element of those heads' dQ and of
+    dK, dV."""
+    B, H, N, d = 4, 16, 2048, 128
+    inp = inputs(B, H, H, N, d, 2048)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = ea.forward(q, k, v, causal=True)
+    dq, dk, dv = ea.backward(q, k, v, o, lse, do, causal=True)
+    torch.cuda.synchronize()
+    for b, h in ((0, 0), (1, 7), (2, 15), (3, 3)):
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        ref = attention_bwd_ref(*(inp[n][sl].double().numpy() for n in ("q", "k", "v", "do")), True, 0,
+                                d ** -0.5)
+        compare((dq[sl], dk[sl], dv[sl]), ref, f"b{b} h{h}")
+
+
+def test_deterministic_and_dk_sums_to_zero():
+    B, Hq, Hkv, N, d = 2, 4, 2, 600, 128
+    inp = inputs(B, Hq, Hkv, N, d, 77)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = ea.forward(q, k, v, causal=True)
+    a = ea.backward(q, k, v, o, lse, do, causal=True)
+    b = ea.backward(q, k, v, o, lse, do, causal=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    dk = a[1].double()
+    # rows of dS sum to zero: sum over keys of dK is ~0 relative to its terms
+    assert (dk.sum(dim=1).abs().max() / dk.abs().sum(dim=1).max()).item() < 2e-2

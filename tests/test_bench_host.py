@@ -203,3 +203,22 @@ def test_pairs_for_rows_with_ranges_brute_force():
                     if lo[i] <= j < hi[i] and (not causal or j <= i) and (window <= 0 or j > i - window):
                         want += 1
             assert bench.pairs_for_rows(rows, N, causal, window, lo, hi) == want
+
+
+def test_reference_arm_on_a_backward_workload():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+           "bwd_bf16_causal_b4h16_n2048_d128", "--steps", "3", "--warmup", "3", "--ref-seconds", "3"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr
+    lines = [l for l in proc.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["metric"].startswith("attention bwd") and j["value"] > 0
+
+
+def test_backward_accounting():
+    from exact_io_aware_78_b200.inputs import BWD_WORKLOADS
+    w = BWD_WORKLOADS["bwd_bf16_causal_b4h16_n2048_d128"]
+    assert accounting.bwd_flops(w) == pytest.approx(10 * 4 * 16 * 128 * (2048 * 2049 // 2))
+    # Q, K, V, O, dO read; dQ, dK, dV written (bf16); LSE read (fp32)
+    assert accounting.bwd_bytes(w) == 8 * (4 * 2048 * 16 * 128 * 2) + 4 * 16 * 2048 * 4

@@ -27,7 +27,7 @@ def lib(lib_path):
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_get_last_error", "attn_status_string", "attn_set_option", "attn_shutdown",
-         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked"])
+         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked", "attn_bwd"])
 
 
 def test_library_exports_every_declared_symbol(lib_path):
@@ -123,6 +123,37 @@ def call_masked(lib, lo=P, hi=P, **kw):
 ])
 def test_masked_argument_errors(lib, kw, code):
     rc = call_masked(lib, **kw)
+    if code is None:
+        assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
+    else:
+        assert rc == code
+
+
+def call_bwd(lib, ptrs=None, B_=1, Hq=2, Hkv=1, N=128, d=128, causal=1, window=0, scale=0.125, dtype=B.EA_BF16):
+    ptrs = ptrs or {}
+    names = ["q", "k", "v", "o", "lse", "do", "dq", "dk", "dv"]
+    args = [ptrs.get(n, P) for n in names]
+    return lib.attn_bwd(*args, B_, Hq, Hkv, N, d, causal, window, scale, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs={"do": None}), B.EA_EINVAL),
+    (dict(ptrs={"dk": None}), B.EA_EINVAL),
+    (dict(N=0), B.EA_EINVAL),
+    (dict(Hq=3, Hkv=2), B.EA_EINVAL),
+    (dict(causal=5), B.EA_EINVAL),
+    (dict(scale=float("nan")), B.EA_EINVAL),
+    (dict(dtype=11), B.EA_EINVAL),
+    (dict(dtype=B.EA_FP8_E4M3), B.EA_EUNSUPPORTED),
+    (dict(dtype=B.EA_FP32, d=64), B.EA_EUNSUPPORTED),
+    (dict(d=96), B.EA_EUNSUPPORTED),
+    (dict(ptrs={"dq": P + 8}), B.EA_EALIGN),
+    (dict(ptrs={"lse": P + 2}), B.EA_EALIGN),
+    (dict(Hq=1 << 16, Hkv=1 << 16, N=1 << 15), B.EA_EINVAL),
+    (dict(), None),
+])
+def test_backward_argument_errors(lib, kw, code):
+    rc = call_bwd(lib, **kw)
     if code is None:
         assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
     else:
