@@ -16,15 +16,16 @@
 //     key/value head, 128-key tile).  K and V stay in shared memory while the
 //     item walks every query tile of every query head of its group that sees
 //     the key tile.  Per step the tensor core computes S^T = K Q^T and
-//     dP^T = V dO^T into tensor memory; the compute warpgroup (one thread per
-//     key row) forms P^T and dS^T and writes them back over S^T and dP^T
-//     as bf16; the tensor core accumulates dV += P^T dO and dK += dS^T Q in
+//     dP^T = V dO^T into tensor memory; two compute warpgroups (one thread
+//     per key row, half of the query columns each) form P^T and dS^T and
+//     write them back over S^T and dP^T as bf16; the tensor core accumulates dV += P^T dO and dK += dS^T Q in
 //     tensor memory (512 columns: S^T, dP^T, dV, dK).  The group's query
 //     heads accumulate into the same dK, dV: no atomics.
 //   * attn_bwd_dq_sm100: a work item is (batch, query head, 128-row query
 //     tile); Q and dO stay in shared memory while the item walks the K/V
-//     tiles it sees: S = Q K^T and dP = dO V^T into tensor memory, the
-//     compute warpgroup (one thread per query row) forms dS over dP, the
+//     tiles it sees: S = Q K^T and dP = dO V^T into tensor memory, two
+//     compute warpgroups (one thread per query row, half of the key columns
+//     each) form dS over dP, the
 //     tensor core accumulates dQ += dS K.  Recomputing S and dP here instead
 //     of adding dQ from the first kernel with atomics keeps the results
 //     deterministic.
@@ -160,7 +161,7 @@ template <int kD>
 struct BwdCfg {
   using C = KernelCfg<2, kD, kD, kOutBf16>;  // the forward's tile layout and MMA helpers
   static constexpr int kTileBytes = 128 * kD * 2;
-  static constexpr int kThreads = 192;       // warps 0-3 compute, 4 MMA, 5 TMA
+  static constexpr int kThreads = 320;       // warps 0-7 compute (two warpgroups), 8 MMA, 9 TMA
   static constexpr int kResOffset = 0;       // resident pair (K, V) or (Q, dO)
   static constexpr int kStageOffset = 2 * kTileBytes;
   static constexpr int kStatsOffset = kStageOffset + 4 * kTileBytes;  // two stages of two tiles
@@ -298,7 +299,9 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
         if (!ok) break;
       }
       tc_fence_after();
-      mma_pv<C, 0, 2 * kHalf>(tDv, tS, do_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      // A = P^T: query columns 0-63 from words [0, 32), 64-127 from [64, 96)
+      mma_pv<C, 0, kHalf>(tDv, tS, do_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, kHalf, 2 * kHalf>(tDv, tS + 32, do_mn[t], kIdAcc, 1u);
       const bool more = s + 1 < it.steps;
       if (more) {
         ok = bwd_warp_wait(&ctl->st_full[t ^ 1], ((step + 1) >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
@@ -310,7 +313,8 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
       if (!ok) break;
       ph_ds ^= 1u;
       tc_fence_after();
-      mma_pv<C, 0, 2 * kHalf>(tDk, tDp, st_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, 0, kHalf>(tDk, tDp, st_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, kHalf, 2 * kHalf>(tDk, tDp + 32, st_mn[t], kIdAcc, 1u);
       mma_commit_elect(&ctl->st_empty[t]);
       if (more) {
         mma_qk<C, 0>(tDp, v_lo, do_lo[t ^ 1], kIdS);
@@ -326,19 +330,33 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
   __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->drain, 0, ctl, p, kSiteBwdDrain, false));
 }
 
-// Stats of the 128 query rows of a step into shared memory (one per thread).
+// Stats of one query row: (-lse2, D), or (-inf, 0) past N.
 __device__ __forceinline__ float2 load_stats(const BwdParams& p, int b, int h, int q) {
   if (q >= p.N) return make_float2(-CUDART_INF_F, 0.0f);
   return __ldg(p.stats + (static_cast<size_t>(b) * p.Hq + h) * p.N + q);
 }
 
-// Thread = key row j of the tile; columns = the step's 128 query rows.
+// The query head and first query row of step s of a dK/dV item.
+__device__ __forceinline__ void kv_step(const KvItem& it, const BwdParams& p, int s, int& h, int& q0) {
+  const int qspan = it.qt_hi - it.qt_lo;
+  h = it.hkv * p.group + s / qspan;
+  q0 = (it.qt_lo + s % qspan) * 128;
+}
+
+// Two warpgroups; thread = key row j of the tile (warp % 4 picks the lane
+// quadrant), warpgroup g takes the step's query columns [64 g, 64 g + 64).
+// Nothing in the backward reduces over a row (P comes from the saved LSE),
+// so the split needs no exchange; it puts two compute warps on every SMSP.
+// Each warpgroup writes its packed P^T (dS^T) words into its own half of
+// the S^T (dP^T) columns, which it has already read: g = 0 into columns
+// [0, 32), g = 1 into [64, 96) (dP^T: +128).
 template <int kD>
 __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t tmem, int warp, int lane) {
   using G = BwdCfg<kD>;
-  const int r = warp * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem + lane_off + G::kColS, tDp = tmem + lane_off + G::kColDp;
+  const int g = warp >> 2;
+  const int r = (warp & 3) * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tS = tmem + lane_off + G::kColS + 64 * g, tDp = tmem + lane_off + G::kColDp + 64 * g;
   const uint32_t tDv = tmem + lane_off + G::kColA0, tDk = tmem + lane_off + G::kColA1;
   float2* sbuf = reinterpret_cast<float2*>(smem + G::kStatsOffset);
   const float cs = p.scale_log2;
@@ -351,69 +369,78 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
     if (it.steps == 0) {            // no query sees this key tile: zero gradients
       if (j < p.N) {
         const size_t row = ((static_cast<size_t>(it.b) * p.N + j) * p.Hkv + it.hkv) * kD;
-        uint4* a = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dk) + row);
-        uint4* c = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dv) + row);
-        for (int x = 0; x < kD / 8; ++x) a[x] = c[x] = make_uint4(0, 0, 0, 0);
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(g == 0 ? p.dv : p.dk) + row);
+        for (int x = 0; x < kD / 8; ++x) dst[x] = make_uint4(0, 0, 0, 0);
       }
       continue;
     }
-    const int qspan = it.qt_hi - it.qt_lo;
+    // warpgroup 0 fetches each step's stats (one row per thread) a step ahead
+    float2 nxt = make_float2(0.0f, 0.0f);
+    if (g == 0) {
+      int h, q0;
+      kv_step(it, p, 0, h, q0);
+      nxt = load_stats(p, it.b, h, q0 + r);
+    }
     for (int s = 0; s < it.steps; ++s, ++step) {
-      const int h = it.hkv * p.group + s / qspan;
-      const int q0 = (it.qt_lo + s % qspan) * 128;
-      // The step's 128 (-lse2, D) pairs, one per thread, into the buffer of
-      // this step's parity; the four warps meet on an mbarrier (bounded
-      // wait).  A warp that passed this step's barrier knows every warp has
-      // finished the step before, so the buffer it writes next is free.
+      int h, q0;
+      kv_step(it, p, s, h, q0);
+      // The step's (-lse2, D) pairs into the buffer of this step's parity;
+      // all eight warps meet on an mbarrier (bounded wait).  A warp that
+      // passed it knows every warp has finished the step before, so the
+      // buffer written next is free.
       float2* st = sbuf + (step & 1) * 128;
-      st[r] = load_stats(p, it.b, h, q0 + r);
+      if (g == 0) {
+        st[r] = nxt;
+        if (s + 1 < it.steps) {
+          int h1, q1;
+          kv_step(it, p, s + 1, h1, q1);
+          nxt = load_stats(p, it.b, h1, q1 + r);
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->stats_ready[step & 1]);
       if (!__all_sync(0xFFFFFFFFu, bwd_wait(&ctl->stats_ready[step & 1], (step >> 1) & 1u, ctl, p,
                                             kSiteBwdCompStats)))
         return;
-      // visible columns: c >= j - q0 (causal), c < j - q0 + window (window)
-      const int vlo = p.causal ? j - q0 : INT_MIN;
-      const int vhi = p.window > 0 ? j - q0 + p.window : INT_MAX;
-      const bool need_mask = __any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 128);
+      const float2* sg = st + 64 * g;
+      // visible columns of this warpgroup: c >= j - q0 - 64 g (causal), c < j - q0 - 64 g + window
+      const int base = j - q0 - 64 * g;
+      const int vlo = p.causal ? base : INT_MIN;
+      const int vhi = p.window > 0 ? base + p.window : INT_MAX;
+      const bool need_mask = __any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 64);
 
       bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->s_full, ph_s, ctl, p, kSiteBwdCompS));
       if (!ok) return;
       ph_s ^= 1u;
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
         uint32_t* raw = reinterpret_cast<uint32_t*>(x);
         tmem_ld32p(tS + 0, raw);
         tmem_ld32p(tS + 32, raw + 32);
-        tmem_ld32p(tS + 64, raw + 64);
-        tmem_ld32p(tS + 96, raw + 96);
         tmem_wait_ld();
       }
-      // P^T row: p = 2^(s cs - lse2), masked to 0; packed bf16 over S^T.
+      // P^T: p = 2^(s cs - lse2), masked to 0; 32 packed bf16 words.
       {
         const uint64_t cs2 = f2_pack(cs, cs);
+        uint32_t pk[32];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int ii = 0; ii < 32; ++ii) {
-            const int c = h2 * 64 + 2 * ii;
-            const float2 a = st[c], b = st[c + 1];
-            const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, f2_pack(a.x, b.x));
-            float y0, y1;
-            f2_unpack(y, y0, y1);
-            float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-            if (need_mask) {
-              if (c < vlo || c >= vhi) e0 = 0.0f;
-              if (c + 1 < vlo || c + 1 >= vhi) e1 = 0.0f;
-            }
-            x[c] = e0;
-            x[c + 1] = e1;
-            pk[ii] = pack_bf16x2(e0, e1);
+        for (int ii = 0; ii < 32; ++ii) {
+          const int c = 2 * ii;
+          const float2 a = sg[c], b = sg[c + 1];
+          const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, f2_pack(a.x, b.x));
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
+          if (need_mask) {
+            if (c < vlo || c >= vhi) e0 = 0.0f;
+            if (c + 1 < vlo || c + 1 >= vhi) e1 = 0.0f;
           }
-          tmem_st32(tS + 32 * h2, pk);
+          x[c] = e0;
+          x[c + 1] = e1;
+          pk[ii] = pack_bf16x2(e0, e1);
         }
+        tmem_st32(tS, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -424,10 +451,10 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
       if (!ok) return;
       ph_dp ^= 1u;
       tc_fence_after();
-      // dS^T row: p (dp - D), packed bf16 over dP^T, 32 columns at a time
-      // (chunk k's 16 packed words land in columns the loads already read).
+      // dS^T: p (dp - D), packed bf16, 32 columns at a time (chunk k's 16
+      // words land in columns this warpgroup has already read).
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 2; ++k) {
         uint32_t dp[32];
         tmem_ld32(tDp + 32 * k, dp);
         tmem_wait_ld();
@@ -435,8 +462,8 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
           const int c = 32 * k + 2 * ii;
-          const float d0 = x[c] * (__uint_as_float(dp[2 * ii]) - st[c].y);
-          const float d1 = x[c + 1] * (__uint_as_float(dp[2 * ii + 1]) - st[c + 1].y);
+          const float d0 = x[c] * (__uint_as_float(dp[2 * ii]) - sg[c].y);
+          const float d1 = x[c + 1] * (__uint_as_float(dp[2 * ii + 1]) - sg[c + 1].y);
           pk[ii] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tDp + 16 * k, pk);
@@ -446,17 +473,16 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->ds_full);
     }
-    // Epilogue: dV and scale * dK of this key row, bf16.
+    // Epilogue: warpgroup 0 stores dV, warpgroup 1 scale * dK, bf16.
     bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->acc_full, items & 1u, ctl, p, kSiteBwdCompAcc));
     if (!ok) return;
     tc_fence_after();
-    const bool store = j < p.N;
-    const size_t row = ((static_cast<size_t>(it.b) * p.N + j) * p.Hkv + it.hkv) * kD;
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t src = which == 0 ? tDv : tDk;
-      const float f = which == 0 ? 1.0f : p.scale;
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(which == 0 ? p.dv : p.dk) + row);
+    {
+      const bool store = j < p.N;
+      const size_t row = ((static_cast<size_t>(it.b) * p.N + j) * p.Hkv + it.hkv) * kD;
+      const uint32_t src = g == 0 ? tDv : tDk;
+      const float f = g == 0 ? 1.0f : p.scale;
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(g == 0 ? p.dv : p.dk) + row);
 #pragma unroll 1
       for (int cc = 0; cc < kD; cc += 32) {
         uint32_t v[32];
@@ -480,7 +506,7 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
 }
 
 template <int kD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const BwdParams p) {
@@ -498,22 +524,22 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&ctl->s_full, 1);
     mbar_init(&ctl->dp_full, 1);
-    mbar_init(&ctl->s_free, 4);
-    mbar_init(&ctl->p_full, 4);
-    mbar_init(&ctl->ds_full, 4);
+    mbar_init(&ctl->s_free, 8);
+    mbar_init(&ctl->p_full, 8);
+    mbar_init(&ctl->ds_full, 8);
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 4);
-    mbar_init(&ctl->stats_ready[0], 4);
-    mbar_init(&ctl->stats_ready[1], 4);
+    mbar_init(&ctl->acc_empty, 8);
+    mbar_init(&ctl->stats_ready[0], 8);
+    mbar_init(&ctl->stats_ready[1], 8);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0) {
+  if (warp == 9 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -523,9 +549,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  if (warp < 4) {
+  if (warp < 8) {
     dkdv_compute<kD>(p, ctl, smem, tmem, warp, lane);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     dkdv_mma<kD>(p, ctl, smem, tmem);
     __syncwarp();
   } else {
@@ -535,7 +561,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == 8) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------ dQ work items
@@ -663,7 +689,9 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
         if (!ok) break;
       }
       tc_fence_after();
-      mma_pv<C, 0, 8>(tDq, tDp, k_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      // A = dS: key columns 0-63 from words [128, 160), 64-127 from [192, 224)
+      mma_pv<C, 0, 4>(tDq, tDp, k_mn[t], kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, 4, 8>(tDq, tDp + 32, k_mn[t], kIdAcc, 1u);
       mma_commit_elect(&ctl->st_empty[t]);
       if (more) {
         mma_qk<C, 0>(tDp, do_lo, v_lo[t ^ 1], kIdS);
@@ -679,13 +707,16 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
   __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->drain, 0, ctl, p, kSiteBwdDrain, false));
 }
 
-// Thread = query row i of the tile; columns = the step's 128 keys.
+// Two warpgroups; thread = query row i of the tile, warpgroup g takes the
+// step's key columns [64 g, 64 g + 64) and writes its packed dS words into
+// its own half of the dP columns ([128, 160) or [192, 224)).
 template <int kD>
 __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int warp, int lane) {
   using G = BwdCfg<kD>;
-  const int r = warp * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem + lane_off + G::kColS, tDp = tmem + lane_off + G::kColDp;
+  const int g = warp >> 2;
+  const int r = (warp & 3) * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tS = tmem + lane_off + G::kColS + 64 * g, tDp = tmem + lane_off + G::kColDp + 64 * g;
   const uint32_t tDq = tmem + lane_off + G::kColA0;
   const float cs = p.scale_log2;
   uint32_t items = 0, ph_s = 0, ph_dp = 0;
@@ -698,19 +729,17 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
     const int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;  // visible keys [key_lo, key_hi)
     const int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
     for (int kt = it.kt_lo; kt < it.kt_hi; ++kt) {
-      const int kbase = kt * 128;
-      const bool need_mask = __any_sync(0xFFFFFFFFu, kbase < key_lo || kbase + 128 > key_hi);
+      const int kbase = kt * 128 + 64 * g;
+      const bool need_mask = __any_sync(0xFFFFFFFFu, kbase < key_lo || kbase + 64 > key_hi);
       bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->s_full, ph_s, ctl, p, kSiteBwdCompS));
       if (!ok) return;
       ph_s ^= 1u;
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
         uint32_t* raw = reinterpret_cast<uint32_t*>(x);
         tmem_ld32p(tS + 0, raw);
         tmem_ld32p(tS + 32, raw + 32);
-        tmem_ld32p(tS + 64, raw + 64);
-        tmem_ld32p(tS + 96, raw + 96);
         tmem_wait_ld();
       }
       tc_fence_before();
@@ -721,7 +750,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
         const uint64_t nl2 = f2_pack(st.x, st.x);
         const int vlo = key_lo - kbase, vhi = key_hi - kbase;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, nl2);
           float y0, y1;
           f2_unpack(y, y0, y1);
@@ -739,7 +768,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
       ph_dp ^= 1u;
       tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 2; ++k) {
         uint32_t dp[32];
         tmem_ld32(tDp + 32 * k, dp);
         tmem_wait_ld();
@@ -758,6 +787,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->ds_full);
     }
+    // Epilogue: warpgroup g stores dQ columns [g kD/2, (g + 1) kD/2), scaled.
     bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->acc_full, items & 1u, ctl, p, kSiteBwdCompAcc));
     if (!ok) return;
     tc_fence_after();
@@ -765,7 +795,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dq) +
                                           ((static_cast<size_t>(it.b) * p.N + qrow) * p.Hq + it.h) * kD);
 #pragma unroll 1
-    for (int cc = 0; cc < kD; cc += 32) {
+    for (int cc = g * (kD / 2); cc < (g + 1) * (kD / 2); cc += 32) {
       uint32_t v[32];
       tmem_ld32(tDq + cc, v);
       tmem_wait_ld();
@@ -786,7 +816,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
 }
 
 template <int kD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const BwdParams p) {
@@ -804,22 +834,22 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&ctl->s_full, 1);
     mbar_init(&ctl->dp_full, 1);
-    mbar_init(&ctl->s_free, 4);
-    mbar_init(&ctl->p_full, 4);
-    mbar_init(&ctl->ds_full, 4);
+    mbar_init(&ctl->s_free, 8);
+    mbar_init(&ctl->p_full, 8);
+    mbar_init(&ctl->ds_full, 8);
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 4);
-    mbar_init(&ctl->stats_ready[0], 4);
-    mbar_init(&ctl->stats_ready[1], 4);
+    mbar_init(&ctl->acc_empty, 8);
+    mbar_init(&ctl->stats_ready[0], 8);
+    mbar_init(&ctl->stats_ready[1], 8);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0) {
+  if (warp == 9 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -829,9 +859,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  if (warp < 4) {
+  if (warp < 8) {
     dq_compute<kD>(p, ctl, tmem, warp, lane);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     dq_mma<kD>(p, ctl, smem, tmem);
     __syncwarp();
   } else {
@@ -841,7 +871,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == 8) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace ea
