@@ -295,6 +295,7 @@ class BackwardOracleSampler:
         self.w = w
         self.qkv = [inp[n].to(torch.float64).numpy() for n in "qkv"]
         self.do = make_grad_output(w.B, w.N, w.Hq, w.d, w.seed + 3).to(torch.float64).numpy()
+        self.ranges = (None, None) if inp.get("key_lo") is None else (inp["key_lo"].numpy(), inp["key_hi"].numpy())
         self.cursor = 0
 
     def run(self, budget_s: float):
@@ -303,7 +304,7 @@ class BackwardOracleSampler:
 
         w = self.w
         q, k, v = self.qkv
-        pairs = accounting.attended_pairs(w.N, w.causal, w.window)
+        lo, hi = self.ranges
         flops = 0.0
         rows_done = 0
         t0 = time.perf_counter()
@@ -311,8 +312,12 @@ class BackwardOracleSampler:
             b, h = divmod(self.cursor % (w.B * w.Hq), w.Hq)
             self.cursor += 1
             kh = h // w.group
+            lo_b = None if lo is None else lo[b:b + 1]
+            hi_b = None if hi is None else hi[b:b + 1]
             attention_bwd_ref(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, kh:kh + 1], v[b:b + 1, :, kh:kh + 1],
-                              self.do[b:b + 1, :, h:h + 1], w.causal, w.window, w.scale)
+                              self.do[b:b + 1, :, h:h + 1], w.causal, w.window, w.scale, key_lo=lo_b, key_hi=hi_b)
+            pairs = (accounting.attended_pairs(w.N, w.causal, w.window) if lo is None else
+                     accounting.range_pairs(lo_b, hi_b, w.causal, w.window))
             flops += 10.0 * w.d * pairs
             rows_done += w.N
             if time.perf_counter() - t0 >= budget_s:
@@ -533,13 +538,19 @@ def run_backward_cuda(args, w, world, rank, local):
         inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
         inp["do"] = do_full[:, :, q_lo:q_hi].contiguous()
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
-    o, lse = ea.forward(q, k, v, causal=w.causal, window=w.window, scale=w.scale)
+    masked = inp.get("key_lo") is not None
+    key_lo, key_hi = (inp[n].to(dev) for n in ("key_lo", "key_hi")) if masked else (None, None)
+    o, lse = ea.forward(q, k, v, causal=w.causal, window=w.window, scale=w.scale, key_lo=key_lo, key_hi=key_hi)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, w.causal, w.window, w.scale, stream=stream)
+        if masked:
+            ea.attn_bwd_masked(q, k, v, o, lse, do, dq, dk, dv, key_lo, key_hi, w.causal, w.window, w.scale,
+                               stream=stream)
+        else:
+            ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, w.causal, w.window, w.scale, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -575,7 +586,7 @@ def run_backward_cuda(args, w, world, rank, local):
         value = job_tflops(flops, args.steps, world, total_ms)
 
     # e2e: the public call with the step's inputs copied from pinned host memory
-    host_in = [(t, t.cpu().pin_memory()) for t in (q, k, v, o, lse, do)]
+    host_in = [(t, t.cpu().pin_memory()) for t in (q, k, v, o, lse, do) + ((key_lo, key_hi) if masked else ())]
     host_out = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in (dq, dk, dv)]
     e2e_steps = max(3, min(args.steps, 50))
     es = torch.cuda.Event(enable_timing=True)
@@ -632,7 +643,8 @@ def run_backward_cuda(args, w, world, rank, local):
                      "kernel_source_hash": kernel_source_hash("backward"),
                      "note": "achieved over the whole step (stats pass + dK/dV kernel + dQ kernel)"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * 3,
+        # stats pass, dK/dV and dQ kernels; row ranges: + the two tile-table kernels
+        "gpu_launches": args.steps * (5 if masked else 3),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -9,10 +9,10 @@ binding, the seeded input generators and the throughput accounting.
 The library is loaded lazily on the first call, and calls raise if it is
 missing: there is no CPU fallback.
 """
-from ._binding import (AttnError, attn_bwd, attn_fwd, attn_fwd_decode, attn_fwd_masked, attn_get_last_error,
-                       attn_set_option, attn_shutdown, attn_status_string, attn_version, backward, forward,
-                       forward_decode, load_library)
+from ._binding import (AttnError, attn_bwd, attn_bwd_masked, attn_fwd, attn_fwd_decode, attn_fwd_masked,
+                       attn_get_last_error, attn_set_option, attn_shutdown, attn_status_string, attn_version, backward,
+                       forward, forward_decode, load_library)
 
-__all__ = ["AttnError", "attn_bwd", "attn_fwd", "attn_fwd_decode", "attn_fwd_masked", "attn_get_last_error",
+__all__ = ["AttnError", "attn_bwd", "attn_bwd_masked", "attn_fwd", "attn_fwd_decode", "attn_fwd_masked", "attn_get_last_error",
            "attn_set_option", "attn_shutdown", "attn_status_string", "attn_version", "backward", "forward",
            "forward_decode", "load_library"]

@@ -34,6 +34,8 @@ _SIGNATURES = {
                                        ctypes.c_void_p, ctypes.c_void_p]),
     "attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7 + [ctypes.c_float, ctypes.c_int,
                                                                                 ctypes.c_void_p]),
+    "attn_bwd_masked": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7 + [ctypes.c_void_p] * 2
+                        + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "attn_get_last_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -188,6 +190,19 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     """Queue dQ, dK, dV = the backward of attn_fwd (bf16) on `stream`.
     q, o, dout, dq [B,N,Hq,d]; k, v, dk, dv [B,N,Hkv,d]; lse [B,Hq,N] fp32;
     all contiguous CUDA tensors on one device; o and lse from the forward."""
+    _backward_call(q, k, v, o, lse, dout, dq, dk, dv, causal, window, None, None, scale, stream)
+
+
+def attn_bwd_masked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                    dout: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, key_lo: torch.Tensor,
+                    key_hi: torch.Tensor, causal: bool = False, window: int = 0, scale: Optional[float] = None,
+                    stream=None) -> None:
+    """attn_bwd for a forward with per-row key ranges (int32 [B, N] CUDA
+    tensors, the ones given to attn_fwd_masked)."""
+    _backward_call(q, k, v, o, lse, dout, dq, dk, dv, causal, window, key_lo, key_hi, scale, stream)
+
+
+def _backward_call(q, k, v, o, lse, dout, dq, dk, dv, causal, window, key_lo, key_hi, scale, stream):
     lib = load_library()
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, N, H, d]")
@@ -203,25 +218,37 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         raise ValueError("lse must be a contiguous float32 CUDA tensor [B, Hq, N]")
     if len({t.device for t in (q, k, v, o, lse, dout, dq, dk, dv)}) != 1:
         raise ValueError("all tensors must be on one device")
+    if (key_lo is None) != (key_hi is None):
+        raise ValueError("key_lo and key_hi come together")
+    for name, t in (("key_lo", key_lo), ("key_hi", key_hi)):
+        if t is not None and (not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous()
+                              or tuple(t.shape) != (B, N) or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous int32 [B, N] tensor on q's device")
     if scale is None:
         scale = d ** -0.5
     device = q.device
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, d, int(bool(causal)), int(window))
     with torch.cuda.device(device):
-        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
-                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, d, int(bool(causal)),
-                          int(window), float(scale), EA_BF16, _stream_handle(stream, device))
+        if key_lo is None:
+            st = lib.attn_bwd(*ptrs, float(scale), EA_BF16, _stream_handle(stream, device))
+        else:
+            st = lib.attn_bwd_masked(*ptrs, key_lo.data_ptr(), key_hi.data_ptr(), float(scale), EA_BF16,
+                                     _stream_handle(stream, device))
     if st != EA_OK:
-        raise AttnError(st, "attn_bwd")
+        raise AttnError(st, "attn_bwd" if key_lo is None else "attn_bwd_masked")
 
 
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
              dout: torch.Tensor, causal: bool = False, window: int = 0, scale: Optional[float] = None,
-             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Allocate dQ, dK, dV on q's device and run attn_bwd; returns them."""
+             stream=None, key_lo: Optional[torch.Tensor] = None,
+             key_hi: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Allocate dQ, dK, dV on q's device and run attn_bwd (attn_bwd_masked
+    with per-row key ranges); returns them."""
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, window, scale, stream)
+    _backward_call(q, k, v, o, lse, dout, dq, dk, dv, causal, window, key_lo, key_hi, scale, stream)
     return dq, dk, dv
 
 

@@ -50,6 +50,10 @@ struct BwdParams {
   void* dk;             // [B, N, Hkv, d] bf16
   void* dv;             // [B, N, Hkv, d] bf16
   int* err;             // device error word
+  const int* key_lo;    // [B, N] per-row key ranges (range variant only)
+  const int* key_hi;
+  const int2* tile_kv;  // [B, num_tiles]: K/V tiles [x, y) of each query tile (range variant)
+  const int2* tile_q;   // [B, num_tiles]: query tiles [x, y) that see each key tile (range variant)
   int B, Hq, Hkv, N, group;
   int causal, window;
   float scale_log2;     // scale * log2(e)
@@ -165,12 +169,35 @@ struct BwdCfg {
   static constexpr int kResOffset = 0;       // resident pair (K, V) or (Q, dO)
   static constexpr int kStageOffset = 2 * kTileBytes;
   static constexpr int kStatsOffset = kStageOffset + 4 * kTileBytes;  // two stages of two tiles
-  static constexpr int kCtlOffset = kStatsOffset + 2 * 128 * 8;
+  static constexpr int kRangeOffset = kStatsOffset + 2 * 128 * 8;     // per-query key ranges (range variant)
+  static constexpr int kCtlOffset = kRangeOffset + 2 * 128 * 8;
   static constexpr int kSmemBytes = 1024 + kCtlOffset + 1024;
   static constexpr uint32_t kColS = 0, kColDp = 128, kColA0 = 256, kColA1 = 256 + kD;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kD == 64 || kD == 128, "head dim");
 };
+
+// ------------------------------------------- per-key-tile query tiles (ranges)
+// With per-row key ranges, tile_q[b, kt] = the span [x, y) of query tiles
+// whose K/V tile range (tile_kv, from row_range_tiles_kernel) contains key
+// tile kt; (0, 0) when none does.  One thread per (b, kt).
+__global__ void __launch_bounds__(128) key_tile_queries_kernel(const int2* __restrict__ tile_kv, int2* tile_q, int B,
+                                                               int num_tiles) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(B) * num_tiles) return;
+  const int b = static_cast<int>(t / num_tiles);
+  const int kt = static_cast<int>(t - static_cast<long long>(b) * num_tiles);
+  const int2* row = tile_kv + static_cast<size_t>(b) * num_tiles;
+  int lo = INT_MAX, hi = INT_MIN;
+  for (int qt = 0; qt < num_tiles; ++qt) {
+    const int2 e = __ldg(row + qt);
+    if (e.x <= kt && kt < e.y) {
+      lo = min(lo, qt);
+      hi = max(hi, qt + 1);
+    }
+  }
+  tile_q[t] = lo < hi ? make_int2(lo, hi) : make_int2(0, 0);
+}
 
 // ------------------------------------------------------ dK, dV work items
 struct KvItem {
@@ -180,7 +207,9 @@ struct KvItem {
 };
 
 // Items ranked heaviest first: with causal masking the early key tiles are
-// seen by the most query tiles.
+// seen by the most query tiles.  With per-row key ranges the query tiles
+// come from the table the pre-pass kernels built.
+template <bool kRanges>
 __device__ __forceinline__ KvItem kv_item(int w, const BwdParams& p) {
   KvItem it;
   const int bh_count = p.B * p.Hkv;
@@ -188,6 +217,13 @@ __device__ __forceinline__ KvItem kv_item(int w, const BwdParams& p) {
   const int bh = w - it.kt * bh_count;
   it.b = bh / p.Hkv;
   it.hkv = bh - it.b * p.Hkv;
+  if constexpr (kRanges) {
+    const int2 e = __ldg(p.tile_q + static_cast<size_t>(it.b) * p.num_tiles + it.kt);
+    it.qt_lo = e.x;
+    it.qt_hi = e.y;
+    it.steps = it.qt_hi > it.qt_lo ? p.group * (it.qt_hi - it.qt_lo) : 0;
+    return it;
+  }
   it.qt_lo = p.causal ? it.kt : 0;
   it.qt_hi = p.num_tiles;
   if (p.window > 0) {
@@ -200,7 +236,7 @@ __device__ __forceinline__ KvItem kv_item(int w, const BwdParams& p) {
   return it;
 }
 
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dkdv_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                               const CUtensorMap* tm_do, const BwdParams& p, BwdCtl* ctl, uint8_t* smem) {
   using G = BwdCfg<kD>;
@@ -211,7 +247,7 @@ __device__ void dkdv_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const KvItem it = kv_item(w, p);
+    const KvItem it = kv_item<kRanges>(w, p);
     if (it.steps == 0) continue;
     ok = bwd_wait(&ctl->kv_empty, (items & 1u) ^ 1u, ctl, p, kSiteBwdProdKv);
     if (!ok) break;
@@ -254,7 +290,7 @@ __device__ void dkdv_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
 //   dV += P^T(s) dO(s);  S^T(s+1) = K Q(s+1)^T;  dK += dS^T(s) Q(s);  dP^T(s+1) = V dO(s+1)^T
 // S^T(s+1) overwrites the columns holding P^T(s), so it follows the dV
 // product; dP^T(s+1) likewise follows the dK product.
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t tmem) {
   using G = BwdCfg<kD>;
   using C = typename G::C;
@@ -278,7 +314,7 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const KvItem it = kv_item(w, p);
+    const KvItem it = kv_item<kRanges>(w, p);
     if (it.steps == 0) continue;
     ok = bwd_warp_wait(&ctl->kv_full, items & 1u, ctl, p, kSiteBwdMmaKv);
     if (!ok) break;
@@ -336,6 +372,13 @@ __device__ __forceinline__ float2 load_stats(const BwdParams& p, int b, int h, i
   return __ldg(p.stats + (static_cast<size_t>(b) * p.Hq + h) * p.N + q);
 }
 
+// Per-row key range of one query row ((0, 0) past N: no key).
+__device__ __forceinline__ int2 load_range(const BwdParams& p, int b, int q) {
+  if (q >= p.N) return make_int2(0, 0);
+  const size_t ix = static_cast<size_t>(b) * p.N + q;
+  return make_int2(__ldg(p.key_lo + ix), __ldg(p.key_hi + ix));
+}
+
 // The query head and first query row of step s of a dK/dV item.
 __device__ __forceinline__ void kv_step(const KvItem& it, const BwdParams& p, int s, int& h, int& q0) {
   const int qspan = it.qt_hi - it.qt_lo;
@@ -350,7 +393,7 @@ __device__ __forceinline__ void kv_step(const KvItem& it, const BwdParams& p, in
 // Each warpgroup writes its packed P^T (dS^T) words into its own half of
 // the S^T (dP^T) columns, which it has already read: g = 0 into columns
 // [0, 32), g = 1 into [64, 96) (dP^T: +128).
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t tmem, int warp, int lane) {
   using G = BwdCfg<kD>;
   const int g = warp >> 2;
@@ -359,12 +402,13 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
   const uint32_t tS = tmem + lane_off + G::kColS + 64 * g, tDp = tmem + lane_off + G::kColDp + 64 * g;
   const uint32_t tDv = tmem + lane_off + G::kColA0, tDk = tmem + lane_off + G::kColA1;
   float2* sbuf = reinterpret_cast<float2*>(smem + G::kStatsOffset);
+  int2* rbuf = reinterpret_cast<int2*>(smem + G::kRangeOffset);
   const float cs = p.scale_log2;
   uint32_t step = 0, items = 0, ph_s = 0, ph_dp = 0;
   for (int i = 0;; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const KvItem it = kv_item(w, p);
+    const KvItem it = kv_item<kRanges>(w, p);
     const int j = it.kt * 128 + r;  // this thread's key
     if (it.steps == 0) {            // no query sees this key tile: zero gradients
       if (j < p.N) {
@@ -374,12 +418,15 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
       }
       continue;
     }
-    // warpgroup 0 fetches each step's stats (one row per thread) a step ahead
+    // warpgroup 0 fetches each step's stats (one row per thread) a step ahead;
+    // with per-row key ranges also each query row's range
     float2 nxt = make_float2(0.0f, 0.0f);
+    int2 nxt_rng = make_int2(0, 0);
     if (g == 0) {
       int h, q0;
       kv_step(it, p, 0, h, q0);
       nxt = load_stats(p, it.b, h, q0 + r);
+      if constexpr (kRanges) nxt_rng = load_range(p, it.b, q0 + r);
     }
     for (int s = 0; s < it.steps; ++s, ++step) {
       int h, q0;
@@ -389,12 +436,15 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
       // passed it knows every warp has finished the step before, so the
       // buffer written next is free.
       float2* st = sbuf + (step & 1) * 128;
+      int2* rg = rbuf + (step & 1) * 128;
       if (g == 0) {
         st[r] = nxt;
+        if constexpr (kRanges) rg[r] = nxt_rng;
         if (s + 1 < it.steps) {
           int h1, q1;
           kv_step(it, p, s + 1, h1, q1);
           nxt = load_stats(p, it.b, h1, q1 + r);
+          if constexpr (kRanges) nxt_rng = load_range(p, it.b, q1 + r);
         }
       }
       __syncwarp();
@@ -403,11 +453,13 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
                                             kSiteBwdCompStats)))
         return;
       const float2* sg = st + 64 * g;
-      // visible columns of this warpgroup: c >= j - q0 - 64 g (causal), c < j - q0 - 64 g + window
+      const int2* rgg = rg + 64 * g;
+      // visible columns of this warpgroup: c >= j - q0 - 64 g (causal), c < j - q0 - 64 g + window,
+      // and with row ranges key_lo(row c) <= j < key_hi(row c)
       const int base = j - q0 - 64 * g;
       const int vlo = p.causal ? base : INT_MIN;
       const int vhi = p.window > 0 ? base + p.window : INT_MAX;
-      const bool need_mask = __any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 64);
+      const bool need_mask = kRanges || __any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 64);
 
       bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->s_full, ph_s, ctl, p, kSiteBwdCompS));
       if (!ok) return;
@@ -435,6 +487,11 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
           if (need_mask) {
             if (c < vlo || c >= vhi) e0 = 0.0f;
             if (c + 1 < vlo || c + 1 >= vhi) e1 = 0.0f;
+            if constexpr (kRanges) {
+              const int2 r0 = rgg[c], r1 = rgg[c + 1];
+              if (j < r0.x || j >= r0.y) e0 = 0.0f;
+              if (j < r1.x || j >= r1.y) e1 = 0.0f;
+            }
           }
           x[c] = e0;
           x[c + 1] = e1;
@@ -505,7 +562,7 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
   }
 }
 
-template <int kD>
+template <int kD, bool kRanges>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -550,12 +607,12 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   if (warp < 8) {
-    dkdv_compute<kD>(p, ctl, smem, tmem, warp, lane);
+    dkdv_compute<kD, kRanges>(p, ctl, smem, tmem, warp, lane);
   } else if (warp == 8) {
-    dkdv_mma<kD>(p, ctl, smem, tmem);
+    dkdv_mma<kD, kRanges>(p, ctl, smem, tmem);
     __syncwarp();
   } else {
-    if (lane == 0) dkdv_producer<kD>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
+    if (lane == 0) dkdv_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
     __syncwarp();
   }
   tc_fence_before();
@@ -571,6 +628,8 @@ struct QItem {
 };
 
 // Heaviest first: with causal masking the late query tiles see the most keys.
+// With per-row key ranges the K/V tiles come from the forward's tile table.
+template <bool kRanges>
 __device__ __forceinline__ QItem q_item(int w, const BwdParams& p) {
   QItem it;
   const int bh_count = p.B * p.Hq;
@@ -579,13 +638,19 @@ __device__ __forceinline__ QItem q_item(int w, const BwdParams& p) {
   it.qt = p.causal ? p.num_tiles - 1 - rnk : rnk;
   it.b = bh / p.Hq;
   it.h = bh - it.b * p.Hq;
+  if constexpr (kRanges) {
+    const int2 e = __ldg(p.tile_kv + static_cast<size_t>(it.b) * p.num_tiles + it.qt);
+    it.kt_lo = e.x;
+    it.kt_hi = e.y;
+    return it;
+  }
   const int last_row = min(it.qt * 128 + 127, p.N - 1);
   it.kt_hi = p.causal ? last_row / 128 + 1 : p.num_tiles;
   it.kt_lo = p.window > 0 ? max(0, it.qt * 128 - p.window + 1) / 128 : 0;
   return it;
 }
 
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                             const CUtensorMap* tm_do, const BwdParams& p, BwdCtl* ctl, uint8_t* smem) {
   using G = BwdCfg<kD>;
@@ -597,7 +662,8 @@ __device__ void dq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, co
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const QItem it = q_item(w, p);
+    const QItem it = q_item<kRanges>(w, p);
+    if (kRanges && it.kt_hi <= it.kt_lo) continue;  // no key visible to this tile: dQ = 0
     ok = bwd_wait(&ctl->kv_empty, (items & 1u) ^ 1u, ctl, p, kSiteBwdProdKv);
     if (!ok) break;
     ++items;
@@ -637,7 +703,7 @@ __device__ void dq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, co
 //   S(s+1) = Q K(s+1)^T as soon as the compute warps have read S(s);
 //   dQ += dS(s) K(s) once dS(s) is in tensor memory (over dP(s));
 //   dP(s+1) = dO V(s+1)^T after it (it overwrites dS(s)).
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t tmem) {
   using G = BwdCfg<kD>;
   using C = typename G::C;
@@ -658,8 +724,9 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
   for (int i = 0; ok; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const QItem it = q_item(w, p);
+    const QItem it = q_item<kRanges>(w, p);
     const int n = it.kt_hi - it.kt_lo;
+    if (kRanges && n <= 0) continue;
     ok = bwd_warp_wait(&ctl->kv_full, items & 1u, ctl, p, kSiteBwdMmaKv);
     if (!ok) break;
     ok = bwd_warp_wait(&ctl->st_full[step & 1], (step >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
@@ -710,7 +777,7 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
 // Two warpgroups; thread = query row i of the tile, warpgroup g takes the
 // step's key columns [64 g, 64 g + 64) and writes its packed dS words into
 // its own half of the dP columns ([128, 160) or [192, 224)).
-template <int kD>
+template <int kD, bool kRanges>
 __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int warp, int lane) {
   using G = BwdCfg<kD>;
   const int g = warp >> 2;
@@ -723,11 +790,24 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
   for (int i = 0;; ++i) {
     const int w = work_rank(i);
     if (w >= p.num_work) break;
-    const QItem it = q_item(w, p);
+    const QItem it = q_item<kRanges>(w, p);
     const int qrow = it.qt * 128 + r;
+    if (kRanges && it.kt_hi <= it.kt_lo) {  // no row of the tile sees a key: dQ = 0
+      if (qrow < p.N) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dq) +
+                                              ((static_cast<size_t>(it.b) * p.N + qrow) * p.Hq + it.h) * kD);
+        for (int x = g * (kD / 16); x < (g + 1) * (kD / 16); ++x) dst[x] = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
     const float2 st = load_stats(p, it.b, it.h, qrow);
-    const int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;  // visible keys [key_lo, key_hi)
-    const int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
+    int key_hi = p.causal ? min(p.N, qrow + 1) : p.N;  // visible keys [key_lo, key_hi)
+    int key_lo = p.window > 0 ? max(0, qrow - p.window + 1) : 0;
+    if (kRanges && qrow < p.N) {
+      const size_t ix = static_cast<size_t>(it.b) * p.N + qrow;
+      key_lo = max(key_lo, __ldg(p.key_lo + ix));
+      key_hi = min(key_hi, __ldg(p.key_hi + ix));
+    }
     for (int kt = it.kt_lo; kt < it.kt_hi; ++kt) {
       const int kbase = kt * 128 + 64 * g;
       const bool need_mask = __any_sync(0xFFFFFFFFu, kbase < key_lo || kbase + 64 > key_hi);
@@ -815,7 +895,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
   }
 }
 
-template <int kD>
+template <int kD, bool kRanges>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -860,12 +940,12 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   if (warp < 8) {
-    dq_compute<kD>(p, ctl, tmem, warp, lane);
+    dq_compute<kD, kRanges>(p, ctl, tmem, warp, lane);
   } else if (warp == 8) {
-    dq_mma<kD>(p, ctl, smem, tmem);
+    dq_mma<kD, kRanges>(p, ctl, smem, tmem);
     __syncwarp();
   } else {
-    if (lane == 0) dq_producer<kD>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
+    if (lane == 0) dq_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
     __syncwarp();
   }
   tc_fence_before();

@@ -1,14 +1,16 @@
-// attn_bwd: the C entry point of the attention backward (declared in
-// include/exactattn.h), included at the end of exactattn.cu, whose helpers
-// (device_state, check_range, aligned, make_map and the process-wide
-// options) it uses.  Validates the arguments, takes the per-row
-// statistics' space from the library's pool, and launches the three kernels
-// of attn_bwd_kernel.cuh on the caller's stream: the (-lse2, D) pass, the
-// dK/dV kernel and the dQ kernel.
+// attn_bwd, attn_bwd_masked: the C entry points of the attention backward
+// (declared in include/exactattn.h), included at the end of exactattn.cu,
+// whose helpers (device_state, check_range, aligned, make_map and the
+// process-wide options) they use.  They validate the arguments, take the
+// per-row statistics' space (and with per-row key ranges the two tile
+// tables) from the library's pool, and launch the kernels of
+// attn_bwd_kernel.cuh on the caller's stream: with ranges the tile-range
+// pre-pass of the forward and the key-tile table first, then the
+// (-lse2, D) pass, the dK/dV kernel and the dQ kernel.
 
 namespace {
 
-template <int kD>
+template <int kD, bool kRanges>
 int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                     const ea::BwdParams& base, const DeviceState& ds, cudaStream_t stream) {
   using G = ea::BwdCfg<kD>;
@@ -16,9 +18,9 @@ int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(ea::attn_bwd_dkdv_sm100<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(ea::attn_bwd_dkdv_sm100<kD, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              G::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(ea::attn_bwd_dq_sm100<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(ea::attn_bwd_dq_sm100<kD, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              G::kSmemBytes) != cudaSuccess)
       return EA_ELAUNCH;
     attr_done[dev] = true;
@@ -27,20 +29,18 @@ int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   p.num_work = p.B * p.Hkv * p.num_tiles;  // (batch, kv head, key tile)
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
-  ea::attn_bwd_dkdv_sm100<kD><<<grid, G::kThreads, G::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  ea::attn_bwd_dkdv_sm100<kD, kRanges><<<grid, G::kThreads, G::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return EA_ELAUNCH;
   p.num_work = p.B * p.Hq * p.num_tiles;  // (batch, query head, query tile)
   grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
-  ea::attn_bwd_dq_sm100<kD><<<grid, G::kThreads, G::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  ea::attn_bwd_dq_sm100<kD, kRanges><<<grid, G::kThreads, G::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
 }
 
-}  // namespace
-
-extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                        const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
-                        int causal, int window, float scale, int dtype, void* stream_ptr) {
+int backward_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, int window,
+                  const int* key_lo, const int* key_hi, float scale, int dtype, void* stream_ptr) {
   // ---- arguments that need no device
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return EA_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return EA_EINVAL;
@@ -68,6 +68,10 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
       check_range(dout, q_bytes) || check_range(dq, q_bytes) || check_range(dk, kv_bytes) ||
       check_range(dv, kv_bytes) || check_range(lse, static_cast<size_t>(B) * Hq * N * 4))
     return EA_EINVAL;
+  const bool ranges = key_lo != nullptr;
+  if (ranges && (check_range(key_lo, static_cast<size_t>(B) * N * 4) ||
+                 check_range(key_hi, static_cast<size_t>(B) * N * 4)))
+    return EA_EINVAL;
   CUtensorMap tq, tk, tv, tdo;
   if (make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hq, N, B) ||
       make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hkv, N, B) ||
@@ -76,12 +80,29 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     return EA_EINVAL;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
 
-  // ---- per-row statistics (-LSE log2 e, D) in stream-ordered pool scratch
+  // ---- per-row statistics (-LSE log2 e, D), and with row ranges the two
+  // tile tables, in stream-ordered pool scratch
   const long long rows = static_cast<long long>(B) * N * Hq;
-  float2* stats = nullptr;
-  if (cudaMallocFromPoolAsync(reinterpret_cast<void**>(&stats), static_cast<size_t>(rows) * sizeof(float2), ds->pool,
-                              stream) != cudaSuccess)
+  const size_t stats_bytes = static_cast<size_t>(rows) * sizeof(float2);
+  const size_t table_bytes = static_cast<size_t>(B) * num_tiles * sizeof(int2);
+  void* scratch = nullptr;
+  if (cudaMallocFromPoolAsync(&scratch, stats_bytes + (ranges ? 2 * table_bytes : 0), ds->pool, stream) !=
+      cudaSuccess)
     return EA_ENOMEM;
+  float2* stats = static_cast<float2*>(scratch);
+  int2* tile_kv = ranges ? reinterpret_cast<int2*>(static_cast<char*>(scratch) + stats_bytes) : nullptr;
+  int2* tile_q = ranges ? tile_kv + static_cast<size_t>(B) * num_tiles : nullptr;
+  if (ranges) {
+    ea::row_range_tiles_kernel<<<static_cast<unsigned>(B * num_tiles), 128, 0, stream>>>(
+        key_lo, key_hi, tile_kv, N, static_cast<int>(num_tiles), causal, window > 0 ? window : 0);
+    const long long tt = static_cast<long long>(B) * num_tiles;
+    ea::key_tile_queries_kernel<<<static_cast<unsigned>((tt + 127) / 128), 128, 0, stream>>>(
+        tile_kv, tile_q, B, static_cast<int>(num_tiles));
+    if (cudaGetLastError() != cudaSuccess) {
+      cudaFreeAsync(scratch, stream);
+      return EA_ELAUNCH;
+    }
+  }
   const long long threads = rows * (d / 8);
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   if (d == 128)
@@ -109,9 +130,36 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.scale = scale;
     p.num_tiles = static_cast<int>(num_tiles);
     p.timeout_ns = g_timeout_ns;
-    rc = d == 128 ? launch_backward<128>(tq, tk, tv, tdo, p, *ds, stream)
-                  : launch_backward<64>(tq, tk, tv, tdo, p, *ds, stream);
+    p.key_lo = key_lo;
+    p.key_hi = key_hi;
+    p.tile_kv = tile_kv;
+    p.tile_q = tile_q;
+    if (ranges)
+      rc = d == 128 ? launch_backward<128, true>(tq, tk, tv, tdo, p, *ds, stream)
+                    : launch_backward<64, true>(tq, tk, tv, tdo, p, *ds, stream);
+    else
+      rc = d == 128 ? launch_backward<128, false>(tq, tk, tv, tdo, p, *ds, stream)
+                    : launch_backward<64, false>(tq, tk, tv, tdo, p, *ds, stream);
   }
-  cudaFreeAsync(stats, stream);
+  cudaFreeAsync(scratch, stream);
   return rc;
+}
+
+}  // namespace
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                        int causal, int window, float scale, int dtype, void* stream) {
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, window, nullptr, nullptr, scale,
+                       dtype, stream);
+}
+
+extern "C" int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                               int causal, int window, const int32_t* key_lo, const int32_t* key_hi, float scale,
+                               int dtype, void* stream) {
+  if (!key_lo || !key_hi) return EA_EINVAL;
+  if (!aligned(key_lo, 4) || !aligned(key_hi, 4)) return EA_EALIGN;
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, window, key_lo, key_hi, scale,
+                       dtype, stream);
 }

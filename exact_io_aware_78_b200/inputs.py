@@ -78,6 +78,9 @@ BWD_WORKLOADS: Dict[str, Workload] = {
                  description="backward of causal self-attention"),
         Workload("bwd_bf16_gqa_causal_b2h32kv8_n4096_d128", 2, 32, 8, 4096, 128, True, 0, "bf16", 4096,
                  description="backward of grouped-query causal attention"),
+        Workload("bwd_bf16_doccausal_b2h16_n16384_d128", 2, 16, 16, 16384, 128, True, 0, "bf16", 1638,
+                 description="backward of the packed-document mask (per-row key ranges)", mask="documents",
+                 mask_min=512, mask_max=4096),
     ]
 }
 

@@ -177,6 +177,23 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              void* stream);
 
 /*
+ * attn_bwd_masked -- attn_bwd for a forward run by attn_fwd_masked: the same
+ * gradients with the per-row key ranges key_lo / key_hi ([B, N] int32,
+ * device, shared by all heads; row i of batch b sees keys key_lo <= j <
+ * key_hi, intersected with causal and window) as the mask.  Pass the same
+ * ranges as the forward.  Rows that see no key contribute nothing; keys no
+ * row sees get dK = dV = 0.  The per-tile ranges (the forward's tile table
+ * and, for the dK/dV kernel, the span of query tiles that see each key
+ * tile) are computed by two small kernels into pool scratch.
+ * Arguments and errors: those of attn_bwd, plus EA_EINVAL for a NULL range
+ * array or one that is not a device allocation of B*N int32, EA_EALIGN for
+ * one that is not 4-byte aligned.
+ */
+int attn_bwd_masked(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, int window,
+                    const int32_t* key_lo, const int32_t* key_hi, float scale, int dtype, void* stream);
+
+/*
  * attn_get_last_error -- synchronise `stream`, then read and clear the
  * current device's error word.  *device_code receives 0 or the recorded
  * failure kind (1 = wait timed out), *site the pipeline wait that failed

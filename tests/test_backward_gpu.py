@@ -4,13 +4,16 @@ dQ, dK, dV for small shapes (GQA groups, d = 64 and 128, causal and windowed
 masks, ragged N), both with the oracle's own O and LSE fed to the kernels
 (the backward alone) and end to end after the tcgen05 forward; sampled
 checks at a benchmark size; determinism; the invariants of the softmax
-Jacobian (dK sums to zero over the keys of a head)."""
+Jacobian (dK sums to zero over the keys of a head).  With per-row key ranges
+(attn_bwd_masked): documents, prefix-LM and random ranges (empty rows, key
+tiles no row sees), and bit-identity with the causal backward when the
+ranges reproduce the causal mask."""
 import numpy as np
 import pytest
 import torch
 
 import exact_io_aware_78_b200 as ea
-from exact_io_aware_78_b200.inputs import make_grad_output, make_inputs
+from exact_io_aware_78_b200.inputs import make_grad_output, make_inputs, make_row_ranges
 from oracle import attention_bwd_ref, attention_ref
 
 pytestmark = pytest.mark.gpu
@@ -126,3 +129,78 @@ def test_deterministic_and_dk_sums_to_zero():
     dk = a[1].double()
     # rows of dS sum to zero: sum over keys of dK is ~0 relative to its terms
     assert (dk.sum(dim=1).abs().max() / dk.abs().sum(dim=1).max()).item() < 2e-2
+
+
+# ------------------------------------------------------------- row ranges
+def run_ranges(kind, B, Hq, Hkv, N, d, causal, window, mn, mx, seed, end_to_end=False, lo=None, hi=None):
+    inp = inputs(B, Hq, Hkv, N, d, seed)
+    if lo is None:
+        lo, hi = make_row_ranges(kind, B, N, seed + 5, mn, mx)
+    lo = torch.as_tensor(lo, dtype=torch.int32)
+    hi = torch.as_tensor(hi, dtype=torch.int32)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    klo, khi = lo.to(dev), hi.to(dev)
+    scale = d ** -0.5
+    q64, k64, v64, do64 = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    o_ref, l_ref = attention_ref(q64, k64, v64, causal, window, scale, key_lo=lo.numpy(), key_hi=hi.numpy())
+    if end_to_end:
+        o, lse = ea.forward(q, k, v, causal=causal, window=window, scale=scale, key_lo=klo, key_hi=khi)
+    else:
+        o = torch.from_numpy(o_ref).to(torch.bfloat16).to(dev)
+        lse = torch.from_numpy(l_ref).float().to(dev)
+    grads = ea.backward(q, k, v, o, lse, do, causal=causal, window=window, scale=scale, key_lo=klo, key_hi=khi)
+    st, code, site = ea.attn_get_last_error()
+    assert st == 0, f"device error code {code} at wait site {site}"
+    ref = attention_bwd_ref(q64, k64, v64, do64, causal, window, scale, key_lo=lo.numpy(), key_hi=hi.numpy(),
+                            o=o_ref, lse=l_ref)
+    compare(grads, ref, f"{kind} B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} c{int(causal)} w{window} e2e{int(end_to_end)}")
+    return grads, ref
+
+
+RANGE_CASES = [
+    # kind, B, Hq, Hkv, N, d, causal, window, min, max
+    ("documents", 2, 4, 2, 1000, 128, True, 0, 40, 400),
+    ("documents", 1, 2, 2, 700, 64, False, 0, 100, 300),
+    ("prefix", 2, 2, 1, 600, 128, False, 0, 1, 500),
+    ("random", 1, 2, 2, 520, 128, False, 0, 1, 1),
+    ("random", 1, 4, 2, 450, 64, True, 0, 1, 1),
+    ("documents", 1, 2, 1, 900, 128, True, 64, 150, 600),
+]
+
+
+@pytest.mark.parametrize("c", RANGE_CASES, ids=lambda c: "{}_B{}h{}kv{}n{}d{}c{}w{}".format(*c[:8]))
+def test_backward_with_row_ranges(c):
+    run_ranges(*c, seed=7000 + c[4] + c[5])
+
+
+def test_backward_with_row_ranges_end_to_end():
+    run_ranges("documents", 2, 4, 2, 1100, 128, True, 0, 50, 500, seed=7100, end_to_end=True)
+
+
+def test_backward_ranges_unseen_key_tiles_and_empty_query_tiles():
+    """Keys [256, 384) seen by no row (their dK, dV rows are zero), query rows
+    [512, 640) that see no key (their dQ rows are zero, a whole query tile)."""
+    B, H, N, d = 1, 2, 768, 128
+    lo = np.zeros((B, N), np.int64)
+    hi = np.full((B, N), 256, np.int64)
+    hi[0, 384:] = N
+    lo[0, 384:] = 384
+    lo[0, 512:640] = hi[0, 512:640] = 5
+    grads, ref = run_ranges("custom", B, H, H, N, d, False, 0, 0, 0, seed=7200, lo=lo, hi=hi)
+    dq, dk, dv = (g.float().cpu() for g in grads)
+    assert torch.all(dk[:, 256:384] == 0) and torch.all(dv[:, 256:384] == 0)
+    assert torch.all(dq[:, 512:640] == 0)
+
+
+def test_ranges_reproducing_causal_give_the_causal_backward_bitwise():
+    B, H, N, d = 2, 4, 800, 128
+    inp = inputs(B, H, H, N, d, 7300)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = ea.forward(q, k, v, causal=True)
+    a = ea.backward(q, k, v, o, lse, do, causal=True)
+    i = torch.arange(N, dtype=torch.int32).view(1, N).repeat(B, 1)
+    b = ea.backward(q, k, v, o, lse, do, causal=False, key_lo=torch.zeros_like(i).to(dev), key_hi=(i + 1).to(dev))
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

@@ -27,7 +27,7 @@ def lib(lib_path):
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_get_last_error", "attn_status_string", "attn_set_option", "attn_shutdown",
-         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked", "attn_bwd"])
+         "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked", "attn_bwd", "attn_bwd_masked"])
 
 
 def test_library_exports_every_declared_symbol(lib_path):
@@ -154,6 +154,17 @@ def call_bwd(lib, ptrs=None, B_=1, Hq=2, Hkv=1, N=128, d=128, causal=1, window=0
 ])
 def test_backward_argument_errors(lib, kw, code):
     rc = call_bwd(lib, **kw)
+    if code is None:
+        assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
+    else:
+        assert rc == code
+
+
+@pytest.mark.parametrize("lo,hi,code", [(None, P, B.EA_EINVAL), (P, None, B.EA_EINVAL), (P + 2, P, B.EA_EALIGN),
+                                         (P, P, None)])
+def test_backward_masked_argument_errors(lib, lo, hi, code):
+    args = [P] * 9
+    rc = lib.attn_bwd_masked(*args, 1, 2, 1, 128, 128, 1, 0, lo, hi, 0.125, B.EA_BF16, None)
     if code is None:
         assert rc in (B.EA_ECUDA, B.EA_EUNSUPPORTED)
     else:
