@@ -132,7 +132,7 @@ struct BwdCtl {
 };
 static_assert(sizeof(BwdCtl) <= 1024, "control block");
 
-__device__ __noinline__ bool bwd_wait_slow(uint32_t a, uint32_t parity, BwdCtl* ctl, const BwdParams& p, int site,
+__device__ __forceinline__ bool bwd_wait_slow(uint32_t a, uint32_t parity, BwdCtl* ctl, const BwdParams& p, int site,
                                            bool honor_abort) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -165,7 +165,16 @@ template <int kD>
 struct BwdCfg {
   using C = KernelCfg<2, kD, kD, kOutBf16>;  // the forward's tile layout and MMA helpers
   static constexpr int kTileBytes = 128 * kD * 2;
-  static constexpr int kThreads = 320;       // warps 0-7 compute (two warpgroups), 8 MMA, 9 TMA
+  // Warps 0-7 compute (two warpgroups), warp 8 issues MMAs, warp 9 TMA,
+  // warps 10-11 only complete warpgroup 2.  setmaxnreg gives the compute
+  // warpgroups 216 registers and warpgroup 2 72: 256 * 216 + 128 * 72 =
+  // 64512 = 384 * 168, the launch budget.
+  static constexpr int kThreads = 384;
+  static constexpr int kLaunchRegs = 168;
+  static constexpr int kComputeRegs = 216;
+  static constexpr int kControlRegs = 72;
+  static_assert(256 * kComputeRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split over budget");
+  static_assert(kThreads * kLaunchRegs <= 65536, "launch register budget");
   static constexpr int kResOffset = 0;       // resident pair (K, V) or (Q, dO)
   static constexpr int kStageOffset = 2 * kTileBytes;
   static constexpr int kStatsOffset = kStageOffset + 4 * kTileBytes;  // two stages of two tiles
@@ -563,7 +572,7 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
 }
 
 template <int kD, bool kRanges>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const BwdParams p) {
@@ -607,13 +616,17 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   if (warp < 8) {
+    regs_increase<G::kComputeRegs>();
     dkdv_compute<kD, kRanges>(p, ctl, smem, tmem, warp, lane);
-  } else if (warp == 8) {
-    dkdv_mma<kD, kRanges>(p, ctl, smem, tmem);
-    __syncwarp();
   } else {
-    if (lane == 0) dkdv_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
-    __syncwarp();
+    regs_decrease<G::kControlRegs>();
+    if (warp == 8) {
+      dkdv_mma<kD, kRanges>(p, ctl, smem, tmem);
+      __syncwarp();
+    } else if (warp == 9) {
+      if (lane == 0) dkdv_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
+      __syncwarp();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -896,7 +909,7 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
 }
 
 template <int kD, bool kRanges>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const BwdParams p) {
@@ -940,13 +953,17 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   if (warp < 8) {
+    regs_increase<G::kComputeRegs>();
     dq_compute<kD, kRanges>(p, ctl, tmem, warp, lane);
-  } else if (warp == 8) {
-    dq_mma<kD, kRanges>(p, ctl, smem, tmem);
-    __syncwarp();
   } else {
-    if (lane == 0) dq_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
-    __syncwarp();
+    regs_decrease<G::kControlRegs>();
+    if (warp == 8) {
+      dq_mma<kD, kRanges>(p, ctl, smem, tmem);
+      __syncwarp();
+    } else if (warp == 9) {
+      if (lane == 0) dq_producer<kD, kRanges>(&tm_q, &tm_k, &tm_v, &tm_do, p, ctl, smem);
+      __syncwarp();
+    }
   }
   tc_fence_before();
   __syncthreads();

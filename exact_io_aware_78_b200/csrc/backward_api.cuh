@@ -23,6 +23,13 @@ int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
         cudaFuncSetAttribute(ea::attn_bwd_dq_sm100<kD, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              G::kSmemBytes) != cudaSuccess)
       return EA_ELAUNCH;
+    // The warpgroups re-split the registers the block is launched with
+    // (setmaxnreg); a block launched with fewer would wait there forever.
+    cudaFuncAttributes a1, a2;
+    if (cudaFuncGetAttributes(&a1, ea::attn_bwd_dkdv_sm100<kD, kRanges>) != cudaSuccess ||
+        cudaFuncGetAttributes(&a2, ea::attn_bwd_dq_sm100<kD, kRanges>) != cudaSuccess ||
+        a1.numRegs < G::kLaunchRegs || a2.numRegs < G::kLaunchRegs)
+      return EA_ELAUNCH;
     attr_done[dev] = true;
   }
   ea::BwdParams p = base;
