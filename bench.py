@@ -45,7 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = {
     "prefill": ["exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh",
                 "exact_io_aware_78_b200/csrc/exactattn.cu"],
-    "decode": ["exact_io_aware_78_b200/csrc/decode_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_api.cuh",
+    "decode": ["exact_io_aware_78_b200/csrc/decode_tc_kernel.cuh", "exact_io_aware_78_b200/csrc/decode_kernel.cuh",
+               "exact_io_aware_78_b200/csrc/decode_api.cuh", "exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh",
                "exact_io_aware_78_b200/csrc/sm100_ptx.cuh"],
     "backward": ["exact_io_aware_78_b200/csrc/attn_bwd_kernel.cuh", "exact_io_aware_78_b200/csrc/backward_api.cuh",
                  "exact_io_aware_78_b200/csrc/attn_fwd_kernel.cuh", "exact_io_aware_78_b200/csrc/sm100_ptx.cuh"],

@@ -41,10 +41,11 @@
 #include <math_constants.h>
 
 #include "sm100_ptx.cuh"
+#include "decode_tc_kernel.cuh"  // the tensor-core key-range kernel (decode_tc_kernel)
 
 namespace ea {
 
-constexpr int kDecodeMaxRows = 8;     // g * Nq query rows per (b, kv head)
+constexpr int kDecodeMaxRows = 8;     // g * Nq query rows per (b, kv head) of the CUDA-core kernel
 constexpr int kDecodeWarps = 4;       // warps per block
 
 struct DecodeParams {

@@ -287,11 +287,16 @@ int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float*
  * Arguments and layout (all device pointers, d contiguous, caller-owned):
  *   q    [B, Nq, Hq, d]  bf16        o    [B, Nq, Hq, d]  bf16 (written)
  *   k, v [B, Nk, Hkv, d] bf16        lse  [B, Hq, Nq]     fp32 (written, natural log)
- *   dtype must be EA_BF16; d is 64 or 128; (Hq / Hkv) * Nq <= 8 query rows
- *   per key/value head (larger query blocks: use attn_fwd).
- *   num_splits: key ranges per (batch, key/value head); 0 chooses enough for
- *   about 16 warps per SM.  Results for different split counts agree within
- *   rounding; a given split count is deterministic.
+ *   dtype must be EA_BF16; d is 64 or 128; (Hq / Hkv) * Nq <= 32 query rows
+ *   per key/value head (<= 8 with num_splits > 0; larger query blocks: use
+ *   attn_fwd).
+ *   num_splits: 0 (recommended) runs the tensor-core kernel: one persistent
+ *   CTA per SM, the K/V tiles of all (batch, key/value head) pairs split
+ *   into equal contiguous ranges, each pair's query rows in the first rows
+ *   of a 128-row tcgen05 tile; > 0 runs the CUDA-core kernel with that many
+ *   key ranges per (batch, key/value head).  Results of the two kernels and
+ *   of different split counts agree within rounding; each is deterministic
+ *   for given sizes.
  *   stream: cudaStream_t (NULL = default stream); the call is asynchronous.
  *
  * Memory: the partial results (per range and query row: 2 + d floats) come
@@ -302,8 +307,8 @@ int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float*
  * pointers, non-positive sizes, Nq > Nk, Hq not a multiple of Hkv, causal not
  * 0/1, a non-positive or non-finite scale, an unknown dtype, negative
  * num_splits, or a buffer that is not one device allocation large enough;
- * EA_EUNSUPPORTED for fp8/fp32 inputs, d other than 64/128, or more than 8
- * query rows per key/value head; EA_EALIGN unless q, k, v, o are 16-byte and
+ * EA_EUNSUPPORTED for fp8/fp32 inputs, d other than 64/128, or more query
+ * rows per key/value head than the chosen kernel takes; EA_EALIGN unless q, k, v, o are 16-byte and
  * lse 4-byte aligned; EA_ENOMEM when the pool cannot supply the partials;
  * EA_ECUDA without a usable sm_100 device; EA_ELAUNCH if a launch fails.
  */

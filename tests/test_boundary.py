@@ -206,7 +206,9 @@ def call_decode(lib, q=P, k=P, v=P, o=P, lse=P, B_=1, Hq=8, Hkv=2, Nq=1, Nk=4096
     (dict(dtype=B.EA_FP8_E4M3), B.EA_EUNSUPPORTED),
     (dict(dtype=B.EA_FP32), B.EA_EUNSUPPORTED),
     (dict(d=96), B.EA_EUNSUPPORTED),
-    (dict(Hq=16, Hkv=2, Nq=2), B.EA_EUNSUPPORTED),       # 16 query rows per KV head > 8
+    (dict(Hq=16, Hkv=2, Nq=2, splits=3), B.EA_EUNSUPPORTED),   # 16 rows per KV head > 8 (CUDA-core kernel)
+    (dict(Hq=16, Hkv=1, Nq=3), B.EA_EUNSUPPORTED),             # 48 rows per KV head > 32 (tensor-core kernel)
+    (dict(Hq=16, Hkv=2, Nq=2), None),                          # 16 rows: the tensor-core kernel takes them
     (dict(o=P + 8), B.EA_EALIGN),
     (dict(lse=P + 2), B.EA_EALIGN),
     (dict(), None),                                       # valid: reaches the device step

@@ -1,5 +1,7 @@
 """Parity of the decode / split-KV forward (attn_fwd_decode, through the C
-ABI) with the float64 oracle attention_kv_ref, on seeded bf16 inputs:
+ABI: the tensor-core kernel for num_splits = 0, the CUDA-core kernel for an
+explicit split count) with the float64 oracle attention_kv_ref, on seeded
+bf16 inputs:
 small shapes covering GQA groups, d = 64 and 128, causal and windowed masks,
 ragged key counts, a single key, Nq > 1 (new tokens causal among
 themselves) and explicit split counts from one to more ranges than key
@@ -65,6 +67,11 @@ CASES = [
     (1, 4, 1, 2, 700, 128, True, 1, 0),      # window 1: each query sees only itself
     (1, 4, 2, 4, 4, 128, True, 0, 0),        # Nq == Nk: self-attention of a short sequence
     (1, 2, 2, 3, 3, 128, False, 0, 2),
+    # tensor-core kernel only (more than 8 rows per kv head), ragged stream-K ranges
+    (2, 16, 1, 2, 1500, 128, True, 0, 0),    # 32 rows per kv head
+    (3, 12, 2, 3, 777, 64, True, 0, 0),      # 18 rows, d = 64
+    (1, 8, 1, 4, 300, 128, True, 100, 0),    # 32 rows, window
+    (4, 32, 8, 1, 16500, 128, False, 0, 0),  # many pairs, ragged last tile
 ]
 
 
@@ -82,6 +89,16 @@ def test_workloads_full_size(lib, name):
     inp = decode_workload_inputs(w)
     o, lse = run(inp, w.causal, w.window)
     check(inp, o, lse, w.causal, w.window, name)
+
+
+def test_tensor_core_and_cuda_core_kernels_agree(lib):
+    """The two key-range kernels compute the same rows (within rounding)."""
+    inp = make_decode_inputs(2, 8, 2, 2, 3000, 128, seed=41)
+    a_o, a_l = run(inp, True, 0, 0)
+    b_o, b_l = run(inp, True, 0, 5)
+    check(inp, a_o, a_l, True, 0, "tensor-core kernel")
+    assert (a_o.float() - b_o.float()).abs().max().item() <= 1.6e-2
+    assert (a_l - b_l).abs().max().item() <= 1e-4
 
 
 def test_split_counts_agree_and_runs_repeat(lib):
