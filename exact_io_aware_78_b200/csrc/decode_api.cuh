@@ -36,11 +36,13 @@ static int decode_tc_launch(const void* q, const void* k, const void* v, void* o
   const long long pairs = static_cast<long long>(B) * Hkv;
   const long long total = pairs * tpp;
   const long long G = std::min<long long>(ds->num_sms, total);
-  // slots per pair: the most CTAs whose ranges touch one pair
+  // slots per pair: four (one per softmax warp) for each of the most CTAs
+  // whose ranges touch one pair
   auto owner = [&](long long x) { return ((x + 1) * G - 1) / total; };
   long long kmax = 1;
   for (long long pr = 0; pr < pairs; ++pr)
     kmax = std::max(kmax, owner((pr + 1) * tpp - 1) - owner(pr * tpp) + 1);
+  kmax *= 4;
   if (pairs * kmax * rows >= (1LL << 31)) return EA_EINVAL;
 
   CUtensorMap tq, tk, tv;
@@ -93,7 +95,7 @@ static int decode_tc_launch(const void* q, const void* k, const void* v, void* o
   int rc = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? EA_OK
                                                                                                    : EA_ELAUNCH;
   if (rc == EA_OK) {
-    kern<<<static_cast<unsigned>(G), 96, smem, stream>>>(tq, tk, tv, tp);
+    kern<<<static_cast<unsigned>(G), 192, smem, stream>>>(tq, tk, tv, tp);
     const unsigned comb_blocks = static_cast<unsigned>((pairs * rows + ea::kDecodeWarps - 1) / ea::kDecodeWarps);
     if (cudaGetLastError() == cudaSuccess) {
       if (d == 128)

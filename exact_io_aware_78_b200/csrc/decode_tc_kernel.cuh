@@ -12,21 +12,29 @@
 // Design.  A decode step is bound by reading K and V once; the arithmetic is
 // ~4 FLOP per byte.  The g * Nq query rows of a key/value head fill the first
 // rows of one 128-row tcgen05 tile (the rest stay zero), so S = Q K^T and
-// O += P V each cost 8 MMAs per 128-key tile -- a quarter of the tile's HBM
-// time -- and one warp's softmax over <= 32 rows keeps up with the stream.
+// O += P V each cost 8 MMAs per 128-key tile -- a third of the tile's HBM
+// time.  The rows are written into all four 32-lane quadrants of the tile,
+// so that four softmax warps (one per SMSP) can each own a quarter of a
+// tile's keys.
 //   * 148 persistent CTAs split the whole stream of K/V tiles (all (batch,
 //     key/value head) pairs, each pair's visible tiles in order) into equal
-//     contiguous ranges ("stream-K"); a CTA emits one partial result (m, l,
-//     unnormalised O) per pair its range touches, into that pair's slot k =
-//     the CTA's rank among the pair's contributors.  The pair's last
-//     contributor marks the remaining slots empty.
-//   * Warp 2 issues TMA copies: the pair's query rows as one box of g heads
-//     x Nq rows, then K(j), V(j) into a shared-memory ring.  Warp 1 issues
-//     the MMAs: S(j) into one of two tensor-memory buffers, so S(j + 1) runs
-//     while the softmax works on S(j); O += P(j) V(j) with P read from
-//     tensor memory.  Warp 0 is the softmax: one thread per query row, lazy
-//     rescale of O (only when the tile maximum moves by more than 8 in log2
-//     units), P written as bf16 over its S buffer.
+//     contiguous ranges ("stream-K").  Per pair its range touches, a CTA
+//     emits four partial results (m, l, unnormalised O), one per softmax
+//     warp, into that pair's slots 4 k .. 4 k + 3, k = the CTA's rank among
+//     the pair's contributors; the pair's last contributor marks the
+//     remaining slots empty.  The combine kernel merges them all by their
+//     log-sum-exps, exactly.
+//   * Warp 5 issues TMA copies: the pair's query rows as one box of g heads
+//     x Nq rows into each lane quadrant of the query tile, then K(j), V(j)
+//     into a shared-memory ring.  Warp 4 issues the MMAs: S(j) into one of
+//     two tensor-memory buffers, so S(j + 1) runs while the softmax works on
+//     S(j); O += P(j) V(j) with P read from tensor memory.  Warps 0-3 are
+//     the softmax: warp w, one thread per query row in quadrant w, keeps its
+//     own running maximum and sum over key columns [32 w, 32 w + 32) of
+//     every tile (an independent split of the keys, as the combine expects),
+//     writes P for its columns and zeros elsewhere over its rows' S buffer,
+//     and rescales its own copy of O lazily (only when its maximum moves by
+//     more than 8 in log2 units).
 //   * Every wait is bounded; on expiry the kernel records the site in the
 //     error word, all roles unwind, tensor memory is freed.
 #pragma once
@@ -79,7 +87,7 @@ struct DecodeTcCfg {
   static constexpr int kRingOffset = kTileBytes;
   static constexpr int kCtlOffset = kRingOffset + kStages * kTileBytes;
   static constexpr int kSmemBytes = 1024 + kCtlOffset + 1024;
-  static constexpr int kThreads = 96;  // warp 0 softmax, 1 MMA, 2 TMA
+  static constexpr int kThreads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
   static constexpr uint32_t kColS = 0, kColO = 256;  // S buffers at 0 and 128
   static constexpr float kTau = 8.0f;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -165,10 +173,13 @@ __device__ void dt_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, co
     ok = dt_wait(&ctl->q_empty, (q_n & 1u) ^ 1u, ctl, p, kSiteDtProdQ);
     if (!ok) break;
     ++q_n;
-    mbar_arrive_expect_tx(&ctl->q_full, static_cast<uint32_t>(C::kQChunks * p.rows * 128));
+    mbar_arrive_expect_tx(&ctl->q_full, static_cast<uint32_t>(4 * C::kQChunks * p.rows * 128));
 #pragma unroll
     for (int c = 0; c < C::kQChunks; ++c)
-      tma_load_4d(smem + G::kQOffset + c * C::kChunkBytes, tm_q, &ctl->q_full, c * 64, hkv * p.group, 0, b, pol);
+#pragma unroll
+      for (int quad = 0; quad < 4; ++quad)  // rows 32 quad .. 32 quad + R - 1
+        tma_load_4d(smem + G::kQOffset + c * C::kChunkBytes + quad * 32 * 128, tm_q, &ctl->q_full, c * 64,
+                    hkv * p.group, 0, b, pol);
     for (int j = sg.j0; j < sg.j1 && ok; ++j) {
       const int kt = p.key_tile_lo + j;
 #pragma unroll
@@ -251,13 +262,15 @@ __device__ void dt_mma(const DecodeTcParams& p, DecodeTcCtl* ctl, uint8_t* smem,
   __all_sync(0xFFFFFFFFu, dt_wait(&ctl->drain, 0, ctl, p, kSiteDtDrain, false));
 }
 
-// Warp 0: thread = tile row t (< R valid).  Row t is query head hkv * g +
+// Warp w (0-3): thread = tile row 32 w + t, query row t (< R valid), key
+// columns [32 w, 32 w + 32) of every tile.  Row t is query head hkv * g +
 // t % g at new-token index t / g (the query box is heads-fastest); its
 // partial row is r = (t % g) * Nq + t / g, the combine kernel's order.
 template <int kD>
-__device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t tmem, int lane) {
+__device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t tmem, int warp, int lane) {
   using G = DecodeTcCfg<kD>;
-  const uint32_t tS = tmem + G::kColS, tO = tmem + G::kColO;  // lanes 0-31: this warp's quadrant
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tS = tmem + lane_off + G::kColS, tO = tmem + lane_off + G::kColO;
   const long long end = dt_start(blockIdx.x + 1, p);
   const bool valid = lane < p.rows;
   const int hg = lane % p.group, qi = lane / p.group;
@@ -277,24 +290,20 @@ __device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t t
       if (!__all_sync(0xFFFFFFFFu, dt_wait(&ctl->s_full[bsel], s_use[bsel] & 1u, ctl, p, kSiteDtSoftS))) return;
       ++s_use[bsel];
       tc_fence_after();
-      float x[128];
-      {
-        uint32_t* raw = reinterpret_cast<uint32_t*>(x);
-        const uint32_t a = tS + 128 * bsel;
-        tmem_ld32p(a + 0, raw);
-        tmem_ld32p(a + 32, raw + 32);
-        tmem_ld32p(a + 64, raw + 64);
-        tmem_ld32p(a + 96, raw + 96);
-        tmem_wait_ld();
-      }
-      const int kbase = (p.key_tile_lo + sg.j0 + j) * 128;
+      float x[32];
+      tmem_ld32(tS + 128 * bsel + 32 * warp, *reinterpret_cast<uint32_t(*)[32]>(x));
+      tmem_wait_ld();
+      const int kbase = (p.key_tile_lo + sg.j0 + j) * 128 + 32 * warp;
       const int vlo = key_lo - kbase, vhi = key_hi - kbase;
-      if (__any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 128)) {
+      if (__any_sync(0xFFFFFFFFu, vlo > 0 || vhi < 32)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 32; ++c)
           if (c < vlo || c >= vhi) x[c] = -CUDART_INF_F;
       }
-      const float m_tile = max128(x) * cs;
+      float mx = fmax3(x[0], x[1], x[2]);
+#pragma unroll
+      for (int c = 3; c < 31; c += 2) mx = fmax3(mx, x[c], x[c + 1]);
+      const float m_tile = fmaxf(mx, x[31]) * cs;
       // The previous product O += P(j - 1) V(j - 1) must be complete before O
       // is rescaled; waiting for each product once keeps the phases in step.
       if (j > 0) {
@@ -322,36 +331,42 @@ __device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t t
           tmem_st32(tO + cc, ov);
         }
       }
+      // P over the S buffer: this warp's 16 packed words, zeros elsewhere.
       const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used);
       float sum = 0.0f;
+      uint32_t own[16];
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) {
+        const float e0 = ex2_approx(fmaf(x[2 * ii], cs, neg_ref));
+        const float e1 = ex2_approx(fmaf(x[2 * ii + 1], cs, neg_ref));
+        sum += e0 + e1;
+        own[ii] = pack_bf16x2(e0, e1);
+      }
+      l += sum;
+      uint32_t pk[32];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t pk[32];
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) {
-          const int c = h2 * 64 + 2 * ii;
-          const float e0 = ex2_approx(fmaf(x[c], cs, neg_ref));
-          const float e1 = ex2_approx(fmaf(x[c + 1], cs, neg_ref));
-          sum += e0 + e1;
-          pk[ii] = pack_bf16x2(e0, e1);
+          const int word = 32 * h2 + ii;  // columns 2 word, 2 word + 1
+          pk[ii] = (word >> 4) == warp ? own[word & 15] : 0u;
         }
         tmem_st32(tS + 128 * bsel + 32 * h2, pk);
       }
-      l += sum;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[bsel]);
     }
-    // Epilogue of the segment: this pair's partial in slot k.
+    // Epilogue of the segment: this warp's partial in slot 4 k + w.
     if (!__all_sync(0xFFFFFFFFu, dt_wait(&ctl->o_full, segs & 1u, ctl, p, kSiteDtSoftO))) return;
     if (!__all_sync(0xFFFFFFFFu, dt_wait(&ctl->pv_done, pv_n & 1u, ctl, p, kSiteDtSoftPv))) return;
     ++pv_n;
     tc_fence_after();
     const long long pair_first = static_cast<long long>(sg.pair) * p.tiles_per_pair;
     const int k = static_cast<int>(blockIdx.x - dt_owner(pair_first, p));
-    const size_t slot0 = static_cast<size_t>(sg.pair) * p.kmax;
-    const size_t prow = (slot0 + k) * p.rows + r;
+    const size_t slot0 = static_cast<size_t>(sg.pair) * p.kmax;  // kmax counts the four slots per CTA
+    const size_t prow = (slot0 + 4 * k + warp) * p.rows + r;
 #pragma unroll 1
     for (int cc = 0; cc < kD; cc += 32) {
       uint32_t ov[32];
@@ -374,7 +389,7 @@ __device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t t
     }
     // The pair's last contributor marks the slots after its own empty.
     if (sg.j1 == p.tiles_per_pair && valid) {
-      for (int k2 = k + 1; k2 < p.kmax; ++k2) {
+      for (int k2 = 4 * (k + 1) + warp; k2 < p.kmax; k2 += 4) {
         const size_t e = (slot0 + k2) * p.rows + r;
         p.part_ml[2 * e] = -CUDART_INF_F;
         p.part_ml[2 * e + 1] = 0.0f;
@@ -387,7 +402,7 @@ __device__ void dt_softmax(const DecodeTcParams& p, DecodeTcCtl* ctl, uint32_t t
 }
 
 template <int kD>
-__global__ void __launch_bounds__(96, 1)
+__global__ void __launch_bounds__(192, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeTcParams p) {
   using G = DecodeTcCfg<kD>;
@@ -407,21 +422,21 @@ __global__ void __launch_bounds__(96, 1)
     mbar_init(&ctl->q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->s_full[b], 1);
-      mbar_init(&ctl->p_full[b], 1);
+      mbar_init(&ctl->p_full[b], 4);
     }
     mbar_init(&ctl->pv_done, 1);
     mbar_init(&ctl->o_full, 1);
-    mbar_init(&ctl->o_empty, 1);
+    mbar_init(&ctl->o_empty, 4);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
   fence_proxy_async_smem();
-  if (warp == 1) {
+  if (warp == 4) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 2 && lane == 0) {
+  if (warp == 5 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -430,9 +445,9 @@ __global__ void __launch_bounds__(96, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  if (warp == 0) {
-    dt_softmax<kD>(p, ctl, tmem, lane);
-  } else if (warp == 1) {
+  if (warp < 4) {
+    dt_softmax<kD>(p, ctl, tmem, warp, lane);
+  } else if (warp == 4) {
     dt_mma<kD>(p, ctl, smem, tmem);
     __syncwarp();
   } else {
@@ -442,7 +457,7 @@ __global__ void __launch_bounds__(96, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 4) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace ea
