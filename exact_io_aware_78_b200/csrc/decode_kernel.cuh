@@ -47,6 +47,7 @@ namespace ea {
 
 constexpr int kDecodeMaxRows = 8;     // g * Nq query rows per (b, kv head) of the CUDA-core kernel
 constexpr int kDecodeWarps = 4;       // warps per block
+constexpr int kCombineFast = 16;      // ranges the combine kernel loads all at once
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // [B, Nq, Hq, d]
@@ -304,36 +305,78 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_combine_kernel(const
   // loads that do not wait on any test.
   const size_t base = static_cast<size_t>(bk) * p.splits * p.rows + r;  // range s at base + s * rows
   float M = -CUDART_INF_F;
-  for (int s = lane; s < p.splits; s += 32) {
-    const size_t idx = base + static_cast<size_t>(s) * p.rows;
-    if (p.part_ml[2 * idx + 1] > 0.0f) M = fmaxf(M, p.part_ml[2 * idx]);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
   float L = 0.0f, o[kPerLane];
 #pragma unroll
   for (int c = 0; c < kPerLane; ++c) o[c] = 0.0f;
-  if (M != -CUDART_INF_F) {
-    for (int s0 = 0; s0 < p.splits; s0 += 32) {
-      float w = 0.0f;
-      const int s = s0 + lane;
-      if (s < p.splits) {
-        const size_t idx = base + static_cast<size_t>(s) * p.rows;
-        const float ls = p.part_ml[2 * idx + 1];
-        w = ls > 0.0f ? exp2f(p.part_ml[2 * idx] - M) : 0.0f;
-        L += ls > 0.0f ? ls * w : 0.0f;
-      }
-      const int n = min(32, p.splits - s0);
-#pragma unroll 8
-      for (int t = 0; t < n; ++t) {
-        const float wt = __shfl_sync(0xFFFFFFFFu, w, t);
-        const float* src = p.part_acc + (base + static_cast<size_t>(s0 + t) * p.rows) * kD + lane * kPerLane;
+  if (p.splits <= kCombineFast) {
+    // Up to 16 ranges: every range's accumulator slice is requested at once,
+    // together with the (m, l) pairs, so the row costs about one memory
+    // latency instead of three.
+    float mv = -CUDART_INF_F, lv = 0.0f;
+    if (lane < p.splits) {
+      const size_t idx = base + static_cast<size_t>(lane) * p.rows;
+      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + 2 * idx);
+      mv = ml.x;
+      lv = ml.y;
+    }
+    float a[kCombineFast][kPerLane];
 #pragma unroll
-        for (int c = 0; c < kPerLane; ++c) o[c] += wt * src[c];
+    for (int t = 0; t < kCombineFast; ++t) {
+      if (t < p.splits) {
+        const float* src = p.part_acc + (base + static_cast<size_t>(t) * p.rows) * kD + lane * kPerLane;
+        if constexpr (kPerLane == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          a[t][0] = v.x, a[t][1] = v.y, a[t][2] = v.z, a[t][3] = v.w;
+        } else {
+#pragma unroll
+          for (int c = 0; c < kPerLane; ++c) a[t][c] = src[c];
+        }
       }
     }
+    M = lv > 0.0f ? mv : -CUDART_INF_F;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+    const float w = (lv > 0.0f && M != -CUDART_INF_F) ? exp2f(mv - M) : 0.0f;
+    L = lv > 0.0f ? lv * w : 0.0f;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
+#pragma unroll
+    for (int t = 0; t < kCombineFast; ++t) {
+      const float wt = __shfl_sync(0xFFFFFFFFu, w, t);
+      if (t < p.splits) {
+#pragma unroll
+        for (int c = 0; c < kPerLane; ++c) o[c] += wt * a[t][c];
+      }
+    }
+  } else {  // more ranges: weights first, then the accumulators 32 ranges at a time
+    for (int s = lane; s < p.splits; s += 32) {
+      const size_t idx = base + static_cast<size_t>(s) * p.rows;
+      if (p.part_ml[2 * idx + 1] > 0.0f) M = fmaxf(M, p.part_ml[2 * idx]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+    if (M != -CUDART_INF_F) {
+      for (int s0 = 0; s0 < p.splits; s0 += 32) {
+        float w = 0.0f;
+        const int s = s0 + lane;
+        if (s < p.splits) {
+          const size_t idx = base + static_cast<size_t>(s) * p.rows;
+          const float ls = p.part_ml[2 * idx + 1];
+          w = ls > 0.0f ? exp2f(p.part_ml[2 * idx] - M) : 0.0f;
+          L += ls > 0.0f ? ls * w : 0.0f;
+        }
+        const int n = min(32, p.splits - s0);
+#pragma unroll 8
+        for (int t = 0; t < n; ++t) {
+          const float wt = __shfl_sync(0xFFFFFFFFu, w, t);
+          const float* src = p.part_acc + (base + static_cast<size_t>(s0 + t) * p.rows) * kD + lane * kPerLane;
+#pragma unroll
+          for (int c = 0; c < kPerLane; ++c) o[c] += wt * src[c];
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
+    }
   }
   const float inv = L > 0.0f ? 1.0f / L : 0.0f;
   __nv_bfloat16* dst = p.o + ((static_cast<size_t>(b) * p.Nq + i) * p.Hq + h) * kD + lane * kPerLane;
