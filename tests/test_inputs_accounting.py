@@ -135,3 +135,16 @@ def test_decode_inputs_are_seeded_bf16():
     b = make_decode_inputs(2, 4, 2, 1, 33, 64, seed=3)
     assert all(torch.equal(a[n], b[n]) for n in "qkv")
     assert a["q"].shape == (2, 1, 4, 64) and a["k"].shape == (2, 33, 2, 64) and a["q"].dtype == torch.bfloat16
+
+
+def test_head_shards_keep_the_row_ranges_whole():
+    """Row ranges are shared by all heads: every shard carries them unchanged."""
+    import torch
+    from exact_io_aware_78_b200.inputs import WORKLOADS, head_shard, shard_inputs, workload_inputs
+    w = WORKLOADS["bf16_doccausal_b2h16_n16384_d128"]
+    inp = workload_inputs(w)
+    sw, q_lo, q_hi, kv_lo, kv_hi = head_shard(w, 4, 1)
+    sub = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
+    assert sub["q"].shape[2] == sw.Hq == 4 and sub["k"].shape[2] == sw.Hkv == 4
+    assert torch.equal(sub["key_lo"], inp["key_lo"]) and torch.equal(sub["key_hi"], inp["key_hi"])
+    assert sw.mask == w.mask and sw.mask_min == w.mask_min
