@@ -258,7 +258,9 @@ def attn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.
     """Queue O, LSE for Nq new query rows against Nk >= Nq cached keys on
     `stream`.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], o [B,Nq,Hq,d] bf16,
     lse [B,Hq,Nq] fp32, contiguous CUDA tensors on one device; query row i is
-    the token at position Nk - Nq + i."""
+    the token at position Nk - Nq + i.  num_splits = 0: the tensor-core
+    kernel (up to 32 query rows per kv head); > 0: the CUDA-core kernel with
+    that many key ranges per (batch, kv head) (up to 8 rows)."""
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
         if not t.is_cuda:
