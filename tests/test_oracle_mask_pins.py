@@ -8,7 +8,6 @@ attention with an explicit boolean mask, and the blockwise recurrence.  The
 mutation tests plant plausible slips in the oracle's mask and check that a
 pin catches each.  CPU only."""
 import math
-import sys
 
 import numpy as np
 import pytest
