@@ -1,20 +1,28 @@
 """Benchmark of the exact attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py --peak        (bf16 / e4m3 dense matmul peaks of GPU 0)
 
 One step = one attn_fwd call (every stage of the forward: tile schedule,
 TMA loads, S = Q K^T, online softmax, O += P V, epilogue) over one batch of
 the workload's seeded synthetic inputs, already resident in HBM.  Each step
 is timed with CUDA events on the launching stream; between steps a 256 MiB
-buffer is written to flush the 126 MB L2 (not timed).  Prints one JSON line.
+buffer is written to flush the 126 MB L2 and the SM clock is probed (both
+untimed).  Prints one JSON line.  The default workload is the largest
+one-GPU configuration (bf16 causal + window 4096, N = 16384); its line also
+carries per_config, the throughput-vs-sequence-length curve over all five
+forward configurations (N = 128 ... 16384), each timed the same way.
 Other workloads: decode_* time one attn_fwd_decode call per step (key-range
 and combine kernels); bf16_doccausal_* one attn_fwd_masked call (tile-range
 pre-pass and the range variant of the forward kernel); bwd_* one attn_bwd
 call (stats pass, dK/dV kernel, dQ kernel) after an untimed forward.
 
-Multi-GPU (torchrun): one process per GPU, each runs its own replica of the
-workload (independent problems, no collective on the data path); the
-barrier and the max-over-ranks reduction are the only communication.
+Multi-GPU: one process per GPU.  Under torchrun WORLD_SIZE must equal
+--gpus; without torchrun, --gpus N > 1 relaunches the command as a torchrun
+job of N ranks.  Each rank runs its own replica of the workload
+(independent problems, no collective on the data path) or, with --shard
+heads, its block of the workload's heads; the barrier and the
+max-over-ranks reduction are the only communication.
 """
 from __future__ import annotations
 
@@ -34,9 +42,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_78_b200 import accounting  # noqa: E402
-from exact_io_aware_78_b200.inputs import (BWD_WORKLOADS, DECODE_WORKLOADS, DEFAULT_BENCH_WORKLOAD,  # noqa: E402
-                                           WORKLOADS, decode_workload_inputs, head_shard, make_grad_output,
-                                           shard_inputs, workload_inputs)
+from exact_io_aware_78_b200.inputs import (BWD_WORKLOADS, CURVE_WORKLOADS, DECODE_WORKLOADS,  # noqa: E402
+                                           DEFAULT_BENCH_WORKLOAD, WORKLOADS, decode_workload_inputs, head_shard,
+                                           make_grad_output, shard_inputs, workload_inputs)
 
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16/FP8 peak) vs seq len, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -341,6 +349,7 @@ class BackwardOracleSampler:
 
 def run_reference(args, w, world, rank):
     if rank != 0:
+        print(f"reference arm: rank {rank} of {world} exits without work", file=sys.stderr, flush=True)
         return
     times = []
     flops_done = 0.0
@@ -362,10 +371,11 @@ def run_reference(args, w, world, rank):
               f"{args.steps} steps of ~{per_step_budget:.3g} s, numpy float64 two-pass oracle; "
               f"TFLOP/s counts attended-pair FLOPs")
     line = {
-        "impl": "reference", "metric": METRIC_BWD if is_backward(w) else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC_BWD if is_backward(w) else METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": any_line_config(w, world, args.shard),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -385,41 +395,37 @@ def workload_config(w) -> dict:
 
 
 # ------------------------------------------------------------- CUDA arm
-def run_cuda(args, w, world, rank, local):
-    import exact_io_aware_78_b200 as ea
+PROBE_CYCLES = (50_000, 250_000)
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    ea.load_library()
-    w_job = w
-    inp = workload_inputs(w)
-    if args.shard == "heads":
-        w, q_lo, q_hi, kv_lo, kv_hi = head_shard(w_job, world, rank)
-        inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
-    q, k, v = (inp[n].to(dev) for n in "qkv")
-    scales = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
-    masked = inp.get("key_lo") is not None
-    key_lo, key_hi = (inp[n].to(dev) for n in ("key_lo", "key_hi")) if masked else (None, None)
-    o_dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
-    o = torch.empty((w.B, w.N, w.Hq, w.d), device=dev, dtype=o_dtype)
-    lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
-    def step():
-        if masked:
-            ea.attn_fwd_masked(q, k, v, o, lse, key_lo, key_hi, w.causal, w.window, w.scale, *scales,
-                               stream=stream)
-        else:
-            ea.attn_fwd(q, k, v, o, lse, w.causal, w.window, w.scale, *scales, stream=stream)
+def sm_clock_probe(stream):
+    """Queue an in-stream SM clock measurement: two spin kernels of known
+    SM-clock cycle counts between events.  The difference of their durations
+    cancels the fixed launch cost; returns the three events."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    torch.cuda._sleep(PROBE_CYCLES[0])
+    ev[1].record(stream)
+    torch.cuda._sleep(PROBE_CYCLES[1])
+    ev[2].record(stream)
+    return ev
 
+
+def probe_mhz(ev) -> float:
+    dt_ms = ev[1].elapsed_time(ev[2]) - ev[0].elapsed_time(ev[1])
+    return (PROBE_CYCLES[1] - PROBE_CYCLES[0]) / (dt_ms * 1e3) if dt_ms > 0 else float("nan")
+
+
+def time_steps(step, flush, stream, dev, args, world, rank, local, check_error):
+    """W untimed warm-up steps, then exactly K steps each between CUDA events
+    on the launching stream, L2 flushed (untimed) before each.  After each
+    timed step (outside its events) an SM clock probe runs, so every step has
+    the SM clock it ran at.  Returns (per-step ms, nvidia-smi clock record,
+    per-step probed SM MHz)."""
     for _ in range(args.warmup):
         flush.zero_()
         step()
-    st, code, site = ea.attn_get_last_error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error {code} at site {site} during warm-up")
-
+    check_error("warm-up")
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     sampler = ClockSampler(local) if rank == 0 else None
@@ -429,32 +435,189 @@ def run_cuda(args, w, world, rank, local):
         sampler.start()
         time.sleep(0.3)
     queue_ahead(flush)
+    probes = []
     for i in range(args.steps):
         flush.zero_()
         starts[i].record(stream)
         step()
         ends[i].record(stream)
+        probes.append(sm_clock_probe(stream))
     torch.cuda.synchronize(dev)
     barrier(world)
     clocks = sampler.stop() if sampler else None
-    st, code, site = ea.attn_get_last_error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error {code} at site {site} in the timed region")
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = dist_max(sum(step_ms), world, dev)
-    flops = accounting.flops(w)  # this rank's launch
+    check_error("the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    return step_ms, clocks, [probe_mhz(ev) for ev in probes]
+
+
+def with_probe(clocks, mhz, ms_per_step):
+    """The nvidia-smi record plus the probed SM clock of the timed steps (and
+    the SM cycles per step it implies)."""
+    out = dict(clocks) if clocks else {}
+    m = statistics.median(mhz)
+    out["sm_mhz_probe_median"] = m
+    out["sm_mhz_probe_min"] = min(mhz)
+    out["sm_cycles_per_step"] = ms_per_step * 1e-3 * m * 1e6
+    out["probe"] = "torch.cuda._sleep spin kernels after each timed step (outside its events)"
+    return out
+
+
+def fp8_peak_record():
+    """The e4m3 dense matmul peak measured on a B200 of this machine (committed
+    summary of `python bench.py --peak`), or None."""
+    path = os.path.join(ROOT, "profiles", "peaks_fp8.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        return json.load(f)
+
+
+def prefill_roofline(w, launch_ms, peaks, peak_kind):
+    """Roofline of the attention kernel for one workload: tensor-bound at
+    4*d FLOPs per attended pair against the dense peak of its input format,
+    except the tiny fp32 case, which launch latency bounds (reported as
+    algorithmic GB/s against the copy bandwidth)."""
+    flops = accounting.flops(w)
+    nbytes = accounting.algorithmic_bytes(w)
+    if w.dtype == "fp32" and w.N <= 256:
+        achieved = nbytes / (launch_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": load_traffic(w.name),
+                "peak_source": f"{peak_kind} HBM copy bandwidth (launch-latency bound: 2 launches)",
+                "algorithmic_bytes": nbytes, "kernel_source_hash": kernel_source_hash()}
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    peak, peak_sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    note = f"{peak_kind} bf16 burst (kernel timed alone)"
+    if w.dtype == "fp8":
+        rec = fp8_peak_record()
+        if rec:
+            peak, peak_sustained = rec["fp8_tflops"], rec["fp8_tflops_sustained"]
+            note = "measured e4m3 burst (torch._scaled_mm 8192^3 on a B200 of this pool, profiles/peaks_fp8.json)"
+        else:
+            peak, peak_sustained = 2 * peak, 2 * peak_sustained
+            note = f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 dense ratio)"
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": load_traffic(w.name), "peak_source": note, "peak_sustained": peak_sustained,
+            "frac_sustained": achieved / peak_sustained, "algorithmic_bytes": nbytes,
+            "kernel_source_hash": kernel_source_hash()}
+
+
+def _timing_config(world: int, shard: str) -> dict:
+    return {"l2": "flushed between timed steps (256 MiB write, untimed)",
+            "host": f"{LEAD_FLUSHES} untimed L2 flushes queued before the first timed step",
+            "parallelism": (f"head shards x{world}" if shard == "heads" else
+                            f"replicas x{world}" if world > 1 else "single GPU")}
+
+
+def line_config(w, world: int, shard: str) -> dict:
+    """The `config` object of a forward line; both arms print the same one."""
+    return {**workload_config(w), "flops_per_step": accounting.flops(w),
+            "flops_half_square_per_step": accounting.flops_half_square(w), **_timing_config(world, shard)}
+
+
+def bwd_line_config(w, world: int, shard: str) -> dict:
+    return {**workload_config(w), "pass": "backward", "flops_per_step": accounting.bwd_flops(w),
+            **_timing_config(world, shard)}
+
+
+def decode_line_config(w, world: int, shard: str) -> dict:
+    return {**workload_config(w), "flops_per_step": accounting.decode_flops(w), **_timing_config(world, shard)}
+
+
+def any_line_config(w, world: int, shard: str) -> dict:
+    if is_decode(w):
+        return decode_line_config(w, world, shard)
+    if is_backward(w):
+        return bwd_line_config(w, world, shard)
+    return line_config(w, world, shard)
+
+
+class PrefillProblem:
+    """Device buffers and the step (one attn_fwd, or attn_fwd_masked with
+    per-row key ranges) of one forward workload, this rank's shard of it
+    with --shard heads."""
+
+    def __init__(self, w_job, args, world, rank, dev, stream):
+        import exact_io_aware_78_b200 as ea
+
+        self.w_job = w = w_job
+        inp = workload_inputs(w_job)
+        if args.shard == "heads":
+            w, q_lo, q_hi, kv_lo, kv_hi = head_shard(w_job, world, rank)
+            inp = shard_inputs(inp, q_lo, q_hi, kv_lo, kv_hi)
+        self.w, self.inp = w, inp
+        self.q, self.k, self.v = (inp[n].to(dev) for n in "qkv")
+        self.scales = [None if inp[n + "_scale"] is None else inp[n + "_scale"].to(dev) for n in "qkv"]
+        self.masked = inp.get("key_lo") is not None
+        self.key_lo, self.key_hi = ((inp[n].to(dev) for n in ("key_lo", "key_hi")) if self.masked
+                                    else (None, None))
+        o_dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
+        self.o = torch.empty((w.B, w.N, w.Hq, w.d), device=dev, dtype=o_dtype)
+        self.lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
+        self.stream = stream
+        self.ea = ea
+        # fp32: + the split kernel; row ranges: + the tile-range kernel
+        self.launches = 1 + int(w.dtype == "fp32") + int(self.masked)
+
+    def step(self):
+        w, ea = self.w, self.ea
+        if self.masked:
+            ea.attn_fwd_masked(self.q, self.k, self.v, self.o, self.lse, self.key_lo, self.key_hi, w.causal,
+                               w.window, w.scale, *self.scales, stream=self.stream)
+        else:
+            ea.attn_fwd(self.q, self.k, self.v, self.o, self.lse, w.causal, w.window, w.scale, *self.scales,
+                        stream=self.stream)
+
+    def check_error(self, where):
+        st, code, site = self.ea.attn_get_last_error(self.stream)
+        if st != 0:
+            raise RuntimeError(f"device error {code} at site {site} during {where}")
+
+
+def job_value(pb, args, world, total_ms, steps):
     if args.shard == "heads":
-        value = sharded_tflops(accounting.flops(w_job), args.steps, total_ms)
-    else:
-        value = job_tflops(flops, args.steps, world, total_ms)
+        return sharded_tflops(accounting.flops(pb.w_job), steps, total_ms)
+    return job_tflops(accounting.flops(pb.w), steps, world, total_ms)
+
+
+def curve_entry(pb, args, world, rank, local, dev, flush, peaks, peak_kind):
+    """One point of the throughput-vs-sequence-length curve, timed exactly as
+    the line's own workload (same K, W, flushes and clock probes)."""
+    step_ms, clocks, mhz = time_steps(pb.step, flush, pb.stream, dev, args, world, rank, local, pb.check_error)
+    total_ms = dist_max(sum(step_ms), world, dev)
+    launch_ms = statistics.mean(step_ms)
+    w = pb.w_job
+    entry = {"workload": w.name, "N": w.N, "input_dtype": w.dtype, "value": job_value(pb, args, world, total_ms,
+                                                                                    args.steps),
+             "unit": "TFLOP/s", "ms_per_step": total_ms / args.steps,
+             "roofline": prefill_roofline(pb.w, launch_ms, peaks, peak_kind),
+             "gpu_launches": args.steps * pb.launches,
+             "clocks": with_probe(clocks, mhz, launch_ms)}
+    return entry
+
+
+def run_cuda(args, w, world, rank, local):
+    import exact_io_aware_78_b200 as ea
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peaks, peak_kind = load_peaks()
+    pb = PrefillProblem(w, args, world, rank, dev, stream)
+    step_ms, clocks, mhz = time_steps(pb.step, flush, stream, dev, args, world, rank, local, pb.check_error)
+    total_ms = dist_max(sum(step_ms), world, dev)
+    value = job_value(pb, args, world, total_ms, args.steps)
 
     # e2e: the public API with pinned host buffers, copies inside the timed region
+    inp = pb.inp
     qh, kh, vh = (inp[n].pin_memory() for n in "qkv")
-    host_in = [(q, qh), (k, kh), (v, vh)]
-    if masked:
-        host_in += [(key_lo, inp["key_lo"].pin_memory()), (key_hi, inp["key_hi"].pin_memory())]
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    host_in = [(pb.q, qh), (pb.k, kh), (pb.v, vh)]
+    if pb.masked:
+        host_in += [(pb.key_lo, inp["key_lo"].pin_memory()), (pb.key_hi, inp["key_hi"].pin_memory())]
+    oh = torch.empty(pb.o.shape, dtype=pb.o.dtype).pin_memory()
+    lh = torch.empty(pb.lse.shape, dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
     es = torch.cuda.Event(enable_timing=True)
     ee = torch.cuda.Event(enable_timing=True)
@@ -464,40 +627,40 @@ def run_cuda(args, w, world, rank, local):
         es.record(stream)
         for dst, src in host_in:
             dst.copy_(src, non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
+        pb.step()
+        oh.copy_(pb.o, non_blocking=True)
+        lh.copy_(pb.lse, non_blocking=True)
         ee.record(stream)
         ee.synchronize()
         if i >= 2:
             e2e_ms.append(es.elapsed_time(ee))
     e2e_total = dist_max(sum(e2e_ms), world, dev)
-    if args.shard == "heads":
-        e2e_value = sharded_tflops(accounting.flops(w_job), e2e_steps, e2e_total)
-    else:
-        e2e_value = job_tflops(flops, e2e_steps, world, e2e_total)
+    e2e_value = job_value(pb, args, world, e2e_total, e2e_steps)
     h2d = sum(src.numel() * src.element_size() for _, src in host_in)
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    launch_ms = statistics.mean(step_ms)
+    w_job = pb.w_job
+    top = {"workload": w_job.name, "N": w_job.N, "input_dtype": w_job.dtype, "value": value, "unit": "TFLOP/s",
+           "ms_per_step": total_ms / args.steps, "roofline": prefill_roofline(pb.w, launch_ms, peaks, peak_kind),
+           "gpu_launches": args.steps * pb.launches, "clocks": with_probe(clocks, mhz, launch_ms)}
+    launches = pb.launches
+    del pb, host_in, qh, kh, vh, oh, lh
+
+    # The rest of the curve: every forward configuration, each timed the same way.
+    curve = None
+    if args.curve == "on" or (args.curve == "auto" and w.name == DEFAULT_BENCH_WORKLOAD):
+        curve = []
+        for name in CURVE_WORKLOADS:
+            if name == w.name:
+                curve.append(top)
+                continue
+            other = PrefillProblem(WORKLOADS[name], args, world, rank, dev, stream)
+            curve.append(curve_entry(other, args, world, rank, local, dev, flush, peaks, peak_kind))
+            del other
+            torch.cuda.empty_cache()
 
     if rank != 0:
         return
-    peaks, peak_kind = load_peaks()
-    bf16_peak = peaks["bf16_tflops"]
-    # The timed region runs the launches back to back; when that holds the
-    # GPU at its power cap (clocks.reasons has sw_power_cap) the sustained
-    # GEMM figure is the like-for-like denominator, so both are reported.
-    ratio = 2.0 if w.dtype == "fp8" else 1.0
-    peak = ratio * bf16_peak
-    peak_sustained = ratio * peaks["bf16_tflops_sustained"]
-    if w.dtype == "fp8":
-        peak_note = f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 dense ratio)"
-    else:
-        peak_note = f"{peak_kind} bf16 burst (kernel timed alone)"
-    launch_ms = statistics.mean(step_ms)
-    achieved = flops / (launch_ms * 1e-3) / 1e12
-    traffic = load_traffic(w.name)
-    # fp32: + the split kernel; row ranges: + the tile-range kernel
-    launches_per_step = 1 + int(w.dtype == "fp32") + int(masked)
     line = {
         "metric": METRIC,
         "value": value,
@@ -509,30 +672,21 @@ def run_cuda(args, w, world, rank, local):
         "higher_is_better": True,
         "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None,
-        "dtype": {"bf16": "bf16", "fp8": "e4m3", "fp32": "bf16x3 (fp32 in/out)"}[w.dtype],
+        "dtype": {"bf16": "bf16", "fp8": "e4m3", "fp32": "bf16x3 (fp32 in/out)"}[w_job.dtype],
         "data": "synthetic",
-        "config": {**workload_config(w_job),
-                   "flops_per_step": accounting.flops(w_job),
-                   "flops_half_square_per_step": accounting.flops_half_square(w_job),
-                   "l2": "flushed between timed steps (256 MiB write, untimed)",
-                   "host": f"{LEAD_FLUSHES} untimed L2 flushes queued before the first timed step",
-                   "parallelism": (f"head shards x{world} (rank 0: query heads {w.Hq}, kv heads {w.Hkv})"
-                                   if args.shard == "heads" else
-                                   f"replicas x{world}" if world > 1 else "single GPU")},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
-                     "peak_sustained": peak_sustained, "frac_sustained": achieved / peak_sustained,
-                     "algorithmic_bytes": accounting.algorithmic_bytes(w),
-                     "kernel_source_hash": kernel_source_hash()},
+        "config": line_config(w_job, world, args.shard),
+        "roofline": top["roofline"],
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": clocks,
+        "gpu_launches": args.steps * launches,
+        "clocks": top["clocks"],
     }
+    if curve is not None:
+        line["per_config"] = curve
     if world == 1 and not args.no_cpu_baseline:
-        dt, fl, rows = OracleSampler(w).run(args.cpu_seconds)
+        dt, fl, rows = OracleSampler(w_job).run(args.cpu_seconds)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
                                 "sample": f"{rows} query rows (128-row chunks of consecutive (b,h) heads) of "
-                                          f"{w.name} in {dt:.1f} s, numpy float64 two-pass oracle; TFLOP/s "
+                                          f"{w_job.name} in {dt:.1f} s, numpy float64 two-pass oracle; TFLOP/s "
                                           f"counts attended-pair FLOPs"}
     print(json.dumps(line), flush=True)
 
@@ -568,33 +722,12 @@ def run_backward_cuda(args, w, world, rank, local):
         else:
             ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, w.causal, w.window, w.scale, stream=stream)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    st, code, site = ea.attn_get_last_error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error {code} at site {site} during warm-up")
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    sampler = ClockSampler(local) if rank == 0 else None
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
-    queue_ahead(flush)
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    clocks = sampler.stop() if sampler else None
-    st, code, site = ea.attn_get_last_error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error {code} at site {site} in the timed region")
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    def check_error(where):
+        st, code, site = ea.attn_get_last_error(stream)
+        if st != 0:
+            raise RuntimeError(f"device error {code} at site {site} during {where}")
+
+    step_ms, clocks, mhz = time_steps(step, flush, stream, dev, args, world, rank, local, check_error)
     total_ms = dist_max(sum(step_ms), world, dev)
     flops = accounting.bwd_flops(w)
     if args.shard == "heads":
@@ -647,11 +780,7 @@ def run_backward_cuda(args, w, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {**workload_config(w_job), "pass": "backward", "flops_per_step": accounting.bwd_flops(w_job),
-                   "l2": "flushed between timed steps (256 MiB write, untimed)",
-                   "host": f"{LEAD_FLUSHES} untimed L2 flushes queued before the first timed step",
-                   "parallelism": (f"head shards x{world}" if args.shard == "heads" else
-                                   f"replicas x{world}" if world > 1 else "single GPU")},
+        "config": bwd_line_config(w_job, world, args.shard),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": load_traffic(w.name),
                      "peak_source": f"{peak_kind} bf16 burst (kernel timed alone)",
@@ -663,7 +792,7 @@ def run_backward_cuda(args, w, world, rank, local):
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         # stats pass, dK/dV and dQ kernels; row ranges: + the two tile-table kernels
         "gpu_launches": args.steps * (5 if masked else 3),
-        "clocks": clocks,
+        "clocks": with_probe(clocks, mhz, launch_ms),
     }
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, rows = BackwardOracleSampler(w).run(args.cpu_seconds)
@@ -698,28 +827,12 @@ def run_decode_cuda(args, w, world, rank, local):
     def step():
         ea.attn_fwd_decode(q, k, v, o, lse, w.causal, w.window, w.scale, 0, stream=stream)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    sampler = ClockSampler(local) if rank == 0 else None
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
-    queue_ahead(flush)
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    clocks = sampler.stop() if sampler else None
-    step_ms = [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
+    def check_error(where):
+        st, code, site = ea.attn_get_last_error(stream)
+        if st != 0:
+            raise RuntimeError(f"device error {code} at site {site} during {where}")
+
+    step_ms, clocks, mhz = time_steps(step, flush, stream, dev, args, world, rank, local, check_error)
     total_ms = dist_max(sum(step_ms), world, dev)
     flops = accounting.decode_flops(w)
     if args.shard == "heads":
@@ -775,18 +888,14 @@ def run_decode_cuda(args, w, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(workload_config(w_job), flops_per_step=accounting.decode_flops(w_job),
-                       l2="flushed between timed steps (256 MiB write, untimed)",
-                       host=f"{LEAD_FLUSHES} untimed L2 flushes queued before the first timed step",
-                       parallelism=(f"head shards x{world}" if args.shard == "heads" else
-                                    f"replicas x{world}" if world > 1 else "single GPU")),
+        "config": decode_line_config(w_job, world, args.shard),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": load_traffic(w.name),
                      "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes": nbytes,
                      "kernel_source_hash": kernel_source_hash("decode")},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * 2,  # key-range kernel + combine kernel
-        "clocks": clocks,
+        "clocks": with_probe(clocks, mhz, launch_ms),
     }
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, rows = DecodeOracleSampler(w).run(args.cpu_seconds)
@@ -797,9 +906,102 @@ def run_decode_cuda(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def world_from_env():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+
+
+def resolve_launch(gpus: int, env) -> str:
+    """How to honour --gpus N: "run" in this process (one GPU, or already one
+    rank of a torchrun job of N), "spawn" N ranks from here (N > 1 and no
+    torchrun environment); a torchrun job of another size is an error."""
+    if gpus < 1:
+        raise ValueError("--gpus must be >= 1")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise ValueError(f"--gpus {gpus} but WORLD_SIZE={world}: launch as many ranks as --gpus asks for")
+        return "run"
+    return "spawn" if gpus > 1 else "run"
+
+
+def spawn_ranks(gpus: int) -> int:
+    """Relaunch this command as a torchrun job of `gpus` ranks on this node
+    (one process per GPU, rendezvous on 127.0.0.1); returns its exit code."""
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def measure_peaks(args):
+    """Dense matmul peaks on this GPU for the roofline denominators: torch
+    bf16 matmul and e4m3 torch._scaled_mm (bf16 output, unit scales) at
+    8192^3, best of 10 back-to-back calls (burst) and the mean over about 4 s
+    of back-to-back calls (sustained, under the power cap), with the SM
+    clock sampled during each.  Prints one JSON line."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n = 8192
+    g = torch.Generator(device="cpu")
+    g.manual_seed(88)
+    a = torch.randn(n, n, generator=g).to(dev)
+    b = torch.randn(n, n, generator=g).to(dev)
+    a16, b16 = a.to(torch.bfloat16), b.to(torch.bfloat16)
+    a8 = a.clamp(-448, 448).to(torch.float8_e4m3fn)
+    b8 = b.clamp(-448, 448).to(torch.float8_e4m3fn).t().contiguous().t()  # column-major, as _scaled_mm wants
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    del a, b
+    stream = torch.cuda.current_stream(dev)
+    kinds = {"bf16": lambda: torch.matmul(a16, b16),
+             "fp8": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)}
+    flop = 2.0 * n ** 3
+    out = {"what": "dense matmul peaks, 8192^3", "gpu": torch.cuda.get_device_name(dev)}
+    for name, fn in kinds.items():
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize(dev)
+        best = float("inf")
+        mhz = []
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            ev = sm_clock_probe(stream)
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+            mhz.append(probe_mhz(ev))
+        sampler = ClockSampler(0)
+        sampler.start()
+        t_end = time.perf_counter() + args.peak_seconds
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        calls = 0
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                fn()
+            calls += 20
+            torch.cuda.synchronize(dev)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks = sampler.stop()
+        out[f"{name}_tflops"] = flop / (best * 1e-3) / 1e12
+        out[f"{name}_tflops_sustained"] = flop * calls / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        out[f"{name}_burst_sm_mhz_probe_median"] = statistics.median(mhz)
+        out[f"{name}_sustained_clocks"] = clocks
+    out["fp8_over_bf16_burst"] = out["fp8_tflops"] / out["bf16_tflops"]
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of this node; without a torchrun environment N > 1 relaunches this command as a "
+                         "torchrun job of N ranks")
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_BENCH_WORKLOAD,
@@ -808,18 +1010,34 @@ def main():
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="with several GPUs: each runs its own replica of the workload (weak scaling), or the "
                          "GPUs split the workload's heads (strong scaling; Hkv must divide by the GPU count)")
+    ap.add_argument("--curve", default="auto", choices=["auto", "on", "off"],
+                    help="add per_config: every forward configuration timed the same way (auto: with the "
+                         "default workload)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="host time for the cpu_baseline sample of the CUDA arm")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="total host time budget of the --impl reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--peak", action="store_true",
+                    help="measure the bf16 and e4m3 dense matmul peaks of GPU 0 instead (one JSON line)")
+    ap.add_argument("--peak-seconds", type=float, default=4.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.peak:
+        measure_peaks(args)
+        return
+    try:
+        how = resolve_launch(args.gpus, os.environ)
+    except ValueError as e:
+        ap.error(str(e))
+    if how == "spawn":
+        sys.exit(spawn_ranks(args.gpus))
     w = {**WORKLOADS, **DECODE_WORKLOADS, **BWD_WORKLOADS}[args.workload]
     if args.impl == "reference":
         # host-only: rank 0 times the oracle, other ranks exit without work
-        run_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        world, rank = world_from_env()
+        run_reference(args, w, world, rank)
         return
     world, rank, local = init_dist()
     try:

@@ -14,24 +14,25 @@ template <int kD, bool kRanges>
 int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                     const ea::BwdParams& base, const DeviceState& ds, cudaStream_t stream) {
   using G = ea::BwdCfg<kD>;
-  static bool attr_done[kMaxDevices] = {};
+  static std::atomic<bool> attr_done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr_done[dev]) {
+  const int rc = once_per_device(attr_done, dev, [] {
     if (cudaFuncSetAttribute(ea::attn_bwd_dkdv_sm100<kD, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              G::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(ea::attn_bwd_dq_sm100<kD, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              G::kSmemBytes) != cudaSuccess)
-      return EA_ELAUNCH;
+      return static_cast<int>(EA_ELAUNCH);
     // The warpgroups re-split the registers the block is launched with
     // (setmaxnreg); a block launched with fewer would wait there forever.
     cudaFuncAttributes a1, a2;
     if (cudaFuncGetAttributes(&a1, ea::attn_bwd_dkdv_sm100<kD, kRanges>) != cudaSuccess ||
         cudaFuncGetAttributes(&a2, ea::attn_bwd_dq_sm100<kD, kRanges>) != cudaSuccess ||
         a1.numRegs < G::kLaunchRegs || a2.numRegs < G::kLaunchRegs)
-      return EA_ELAUNCH;
-    attr_done[dev] = true;
-  }
+      return static_cast<int>(EA_ELAUNCH);
+    return static_cast<int>(EA_OK);
+  });
+  if (rc != EA_OK) return rc;
   ea::BwdParams p = base;
   p.num_work = p.B * p.Hkv * p.num_tiles;  // (batch, kv head, key tile)
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -34,6 +35,13 @@ DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 PFN_cuMemGetAddressRange_v3020 g_addr_range = nullptr;
 
+// attn_fwd_fp32_noalloc's per-device set-up: the device address of its
+// static scratch array (looked up by the first call on each device and
+// forgotten by attn_shutdown, which also ends that set-up) and the SM count.
+std::mutex g_noalloc_mutex;
+uint8_t* g_noalloc_ptr[kMaxDevices] = {};
+int g_noalloc_sms[kMaxDevices] = {};
+
 // Options (attn_set_option).
 unsigned long long g_timeout_ns = 2000000000ull;
 int g_max_ctas = 0;
@@ -41,20 +49,44 @@ int g_order = 0;
 int g_skip_arrive_once = 0;
 
 
+// The two driver entry points, looked up once per process (every path that
+// needs them goes through here, so they are published exactly once and read
+// without a lock afterwards).
+std::once_flag g_entry_once;
+int g_entry_rc = EA_ECUDA;
+
 int load_driver_entry_points() {
-  if (g_encode && g_addr_range) return EA_OK;
-  cudaDriverEntryPointQueryResult q1, q2;
-  void* f1 = nullptr;
-  void* f2 = nullptr;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
-      q1 != cudaDriverEntryPointSuccess || f1 == nullptr)
-    return EA_ECUDA;
-  if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
-      q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
-    return EA_ECUDA;
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f1);
-  g_addr_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(f2);
-  return EA_OK;
+  std::call_once(g_entry_once, [] {
+    cudaDriverEntryPointQueryResult q1, q2;
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || f1 == nullptr)
+      return;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+      return;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f1);
+    g_addr_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(f2);
+    g_entry_rc = EA_OK;
+  });
+  return g_entry_rc;
+}
+
+// One-time, per-device set-up of a kernel's launch attributes.  The flag is
+// read without the lock once it is set; the set-up itself runs under a lock,
+// so concurrent first calls on one device perform it once and none launches
+// before it has finished.
+std::mutex g_attr_mutex;
+
+template <class F>
+int once_per_device(std::atomic<bool>* done, int dev, F&& setup) {
+  if (done[dev].load(std::memory_order_acquire)) return EA_OK;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  if (done[dev].load(std::memory_order_relaxed)) return EA_OK;
+  const int rc = setup();
+  if (rc == EA_OK) done[dev].store(true, std::memory_order_release);
+  return rc;
 }
 
 // Per-device state, created on first use with the device current.
@@ -123,21 +155,22 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize
 template <class C, bool kRanges>
 int launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const ea::FwdParams& p,
                    const DeviceState& ds, cudaStream_t stream) {
-  static bool attr_done[kMaxDevices] = {};
+  static std::atomic<bool> attr_done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr_done[dev]) {
+  const int rc = once_per_device(attr_done, dev, [] {
     if (cudaFuncSetAttribute(ea::attn_fwd_sm100<C, kRanges>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
-      return EA_ELAUNCH;
+      return static_cast<int>(EA_ELAUNCH);
     // The warpgroups re-split the registers the block is launched with
     // (setmaxnreg); a block launched with fewer than the split assumes would
     // wait in setmaxnreg forever, so refuse to launch it.
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, ea::attn_fwd_sm100<C, kRanges>) != cudaSuccess || fa.numRegs < C::kLaunchRegs)
-      return EA_ELAUNCH;
-    attr_done[dev] = true;
-  }
+      return static_cast<int>(EA_ELAUNCH);
+    return static_cast<int>(EA_OK);
+  });
+  if (rc != EA_OK) return rc;
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
   ea::attn_fwd_sm100<C, kRanges><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
@@ -289,16 +322,15 @@ int forward_impl(const void* q, const void* k, const void* v, void* o, float* ls
       int pow2 = 1;
       while (pow2 < pairs) pow2 <<= 1;
       const size_t smem = static_cast<size_t>(pow2) * sizeof(unsigned long long);
-      static bool attr_done[kMaxDevices] = {};
+      static std::atomic<bool> attr_done[kMaxDevices];
       int dev = 0;
       cudaGetDevice(&dev);
-      if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(ea::order_items_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 ea::kOrderMaxPairs * static_cast<int>(sizeof(unsigned long long))) != cudaSuccess)
-          rc = EA_ELAUNCH;
-        else
-          attr_done[dev] = true;
-      }
+      rc = once_per_device(attr_done, dev, [] {
+        return cudaFuncSetAttribute(ea::order_items_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ea::kOrderMaxPairs * static_cast<int>(sizeof(unsigned long long))) == cudaSuccess
+                   ? static_cast<int>(EA_OK)
+                   : static_cast<int>(EA_ELAUNCH);
+      });
       if (rc == EA_OK) {
         order = reinterpret_cast<int*>(static_cast<char*>(scratch) + tb);
         ea::order_items_kernel<<<1, 1024, smem, stream>>>(tile_kv, order, static_cast<int>(pairs),
@@ -470,6 +502,15 @@ int attn_set_option(int option, long long value) {
 
 int attn_shutdown(void) {
   std::lock_guard<std::mutex> lock(g_mutex);
+  {
+    // attn_fwd_fp32_noalloc looks its array's address up again on its next
+    // call (the address does not outlive a context the caller may reset).
+    std::lock_guard<std::mutex> nlock(g_noalloc_mutex);
+    for (int dev = 0; dev < kMaxDevices; ++dev) {
+      g_noalloc_ptr[dev] = nullptr;
+      g_noalloc_sms[dev] = 0;
+    }
+  }
   int rc = EA_OK;
   int prev = 0;
   cudaGetDevice(&prev);
@@ -499,17 +540,17 @@ namespace {
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[EA_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mutex;
-uint8_t* g_noalloc_ptr[kMaxDevices] = {};  // device address of the array, per device
-int g_noalloc_sms[kMaxDevices] = {};
-
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Once per device, with that device current: the array's device address
 // (host code must not use the symbol itself as a device pointer).
-int noalloc_setup(int dev) {
+int noalloc_setup(int dev, uint8_t** base, int* num_sms) {
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] != nullptr) return EA_OK;
+  if (g_noalloc_ptr[dev] != nullptr) {
+    *base = g_noalloc_ptr[dev];
+    *num_sms = g_noalloc_sms[dev];
+    return EA_OK;
+  }
   int rc = load_driver_entry_points();
   if (rc != EA_OK) return rc;
   int major = 0, sms = 0;
@@ -525,6 +566,8 @@ int noalloc_setup(int dev) {
     return EA_ECUDA;
   g_noalloc_sms[dev] = sms;
   g_noalloc_ptr[dev] = static_cast<uint8_t*>(ptr);
+  *base = g_noalloc_ptr[dev];
+  *num_sms = sms;
   return EA_OK;
 }
 
@@ -556,7 +599,9 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EA_ECUDA;
   if (dev < 0 || dev >= kMaxDevices) return EA_EUNSUPPORTED;
-  int rc = noalloc_setup(dev);
+  uint8_t* base = nullptr;
+  int num_sms = 0;
+  int rc = noalloc_setup(dev, &base, &num_sms);
   if (rc != EA_OK) return rc;
   const size_t q_bytes = static_cast<size_t>(q_rows) * 64 * 4;
   const size_t kv_bytes = static_cast<size_t>(kv_rows) * 64 * 4;
@@ -566,7 +611,6 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
     return EA_EINVAL;
 
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
-  uint8_t* base = g_noalloc_ptr[dev];
   uint16_t* qs = reinterpret_cast<uint16_t*>(base);
   uint16_t* ks = reinterpret_cast<uint16_t*>(base + sq);
   uint16_t* vs = reinterpret_cast<uint16_t*>(base + sq + sk);
@@ -593,7 +637,7 @@ extern "C" int attn_fwd_fp32_noalloc(const float* q, const float* k, const float
   p.timeout_ns = g_timeout_ns;
 
   DeviceState ds;
-  ds.num_sms = g_noalloc_sms[dev];
+  ds.num_sms = num_sms;
   rc = launch_split({q, qs, q_rows}, {k, ks, kv_rows}, {v, vs, kv_rows}, ds.num_sms, stream);
   if (rc != EA_OK) return rc;
   CUtensorMap tq, tk, tv;

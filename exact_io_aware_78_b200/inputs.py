@@ -67,8 +67,16 @@ WORKLOADS: Dict[str, Workload] = {
     ]
 }
 
-# The workload the benchmark times by default (causal, B=4, H=16, N=2048, d=128).
-DEFAULT_BENCH_WORKLOAD = "bf16_causal_b4h16_n2048_d128"
+# The five forward configurations of the throughput-vs-sequence-length curve,
+# shortest sequence first: fp32 N=128 d=64; bf16 causal N=2048; bf16 GQA
+# causal N=4096 (Q x 3); bf16 causal + window 4096 at N=16384; e4m3 causal
+# N=8192.
+CURVE_WORKLOADS = ("fp32_n128_d64", "bf16_causal_b4h16_n2048_d128", "bf16_gqa_causal_b2h32kv8_n4096_d128_q3",
+                   "bf16_causal_window4096_b1h16_n16384_d128", "fp8_causal_b2h16_n8192_d128")
+
+# The workload the benchmark times by default: the largest one-GPU
+# configuration (causal + sliding window 4096, B=1, H=16, N=16384, d=128).
+DEFAULT_BENCH_WORKLOAD = "bf16_causal_window4096_b1h16_n16384_d128"
 
 # Backward-pass workloads: the forward's inputs plus dO = make_grad_output(seed + 3).
 BWD_WORKLOADS: Dict[str, Workload] = {

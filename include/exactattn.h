@@ -43,9 +43,12 @@
  * recorded in the device error word and reported by attn_get_last_error().
  * No function aborts the process or traps the GPU.
  *
- * Thread safety: calls for different devices may run concurrently; calls
- * for one device are serialised by an internal lock around state creation
- * only, and launches on one stream are ordered by that stream.
+ * Thread safety: calls may come from several host threads.  Creating the
+ * per-device state and the one-time launch set-up of each kernel run under
+ * internal locks (concurrent first calls on a device do them once); after
+ * that, calls take no lock, and launches on one stream are ordered by that
+ * stream.  attn_set_option changes process-wide settings and should not race
+ * with calls; attn_shutdown must not race with any call.
  */
 #ifndef EXACTATTN_H
 #define EXACTATTN_H
@@ -230,7 +233,8 @@ enum {
 int attn_set_option(int option, long long value);
 
 /* attn_shutdown -- free all per-device library state (call after the
- * streams that used it are idle).  Returns EA_OK or EA_ECUDA. */
+ * streams that used it are idle) and forget attn_fwd_fp32_noalloc's
+ * per-device set-up.  Returns EA_OK or EA_ECUDA. */
 int attn_shutdown(void);
 
 /* attn_version -- library ABI version (major * 10000 + minor * 100 + patch). */
@@ -254,7 +258,9 @@ int attn_version(void);
  *             as attn_fwd with dtype EA_FP32 (fp32 in, fp32 O, d == 64).
  *   status    optional device int (NULL allowed): cleared on `stream`, then
  *             set to (kind << 16) | site if a device-side pipeline wait runs
- *             past its limit.  attn_get_last_error does not see this variant.
+ *             past its limit.  attn_get_last_error does not see this variant,
+ *             so without a status word such a timeout goes unreported and the
+ *             outputs of that call are undefined: pass a status word.
  *
  * Scratch needed: 384 * B*N*Hq + 640 * B*N*Hkv bytes (each of the three
  * parts rounded up to 256 bytes) plus 256; a request above
@@ -262,9 +268,11 @@ int attn_version(void);
  * The first call on a device is a set-up call: with that device current it
  * looks up the array's device address (with lazy module loading the CUDA
  * runtime places the array on the device at that point) and synchronises
- * the device once; make that first call before any stream capture.  Every call shares the one array and overwrites it completely
- * before reading it, so calls whose work overlaps on the GPU (different
- * streams, or different host threads) race: serialise them.
+ * the device once; make that first call before any stream capture.
+ * attn_shutdown() forgets that set-up, so the next call on each device is a
+ * set-up call again.  Every call shares the one array and overwrites the part
+ * it uses before reading it, so calls whose work overlaps on the GPU
+ * (different streams, or different host threads) race: serialise them.
  */
 #define EA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 int attn_fwd_fp32_noalloc(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq,

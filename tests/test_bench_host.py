@@ -70,8 +70,8 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_exit_without_work():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2")
-    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "fp32_n128_d64",
-           "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference", "--workload",
+           "fp32_n128_d64", "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
     proc = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert proc.returncode == 0 and proc.stdout.strip() == ""
 
@@ -222,3 +222,66 @@ def test_backward_accounting():
     assert accounting.bwd_flops(w) == pytest.approx(10 * 4 * 16 * 128 * (2048 * 2049 // 2))
     # Q, K, V, O, dO read; dQ, dK, dV written (bf16); LSE read (fp32)
     assert accounting.bwd_bytes(w) == 8 * (4 * 2048 * 16 * 128 * 2) + 4 * 16 * 2048 * 4
+
+
+# ---- --gpus N: the launcher and the shared config object
+
+def test_resolve_launch():
+    assert bench.resolve_launch(1, {}) == "run"
+    assert bench.resolve_launch(4, {}) == "spawn"
+    assert bench.resolve_launch(2, {"WORLD_SIZE": "2"}) == "run"
+    assert bench.resolve_launch(1, {"WORLD_SIZE": "1"}) == "run"
+    with pytest.raises(ValueError):
+        bench.resolve_launch(8, {"WORLD_SIZE": "1"})  # torchrun job of another size
+    with pytest.raises(ValueError):
+        bench.resolve_launch(1, {"WORLD_SIZE": "2"})
+    with pytest.raises(ValueError):
+        bench.resolve_launch(0, {})
+
+
+def test_gpus_mismatch_with_torchrun_is_an_error():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference", "--workload",
+           "fp32_n128_d64", "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert proc.returncode != 0 and "WORLD_SIZE" in proc.stderr
+
+
+def test_gpus_two_spawns_two_ranks_and_prints_one_line():
+    """--gpus 2 without a torchrun environment relaunches the command as a
+    two-rank torchrun job: rank 0 prints the one JSON line with n_gpus 2,
+    rank 1 reports that it exits without work."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                                                          "MASTER_PORT")}
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference", "--workload",
+           "fp32_n128_d64", "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    lines = [l for l in proc.stdout.splitlines() if l.lstrip().startswith("{")]
+    assert len(lines) == 1, proc.stdout
+    j = json.loads(lines[0])
+    assert j["n_gpus"] == 2 and j["impl"] == "reference"
+    assert "rank 1 of 2 exits without work" in proc.stderr
+
+
+@pytest.mark.parametrize("name", ["bf16_causal_window4096_b1h16_n16384_d128", "decode_b4h32kv8_nq2_nk8192_d128_window2048",
+                                  "bwd_bf16_causal_b4h16_n2048_d128"])
+def test_reference_arm_config_is_the_cuda_arms(name):
+    """Both arms print the same `config` object for a workload."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", name,
+           "--steps", "3", "--warmup", "3", "--ref-seconds", "1.5"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    j = json.loads([l for l in proc.stdout.splitlines() if l.lstrip().startswith("{")][0])
+    from exact_io_aware_78_b200.inputs import BWD_WORKLOADS, DECODE_WORKLOADS
+    w = {**WORKLOADS, **DECODE_WORKLOADS, **BWD_WORKLOADS}[name]
+    assert j["config"] == json.loads(json.dumps(bench.any_line_config(w, 1, "replicas")))
+
+
+def test_default_workload_is_the_largest_forward_configuration():
+    from exact_io_aware_78_b200.inputs import CURVE_WORKLOADS, DEFAULT_BENCH_WORKLOAD
+    assert DEFAULT_BENCH_WORKLOAD in CURVE_WORKLOADS and len(CURVE_WORKLOADS) == 5
+    ws = [WORKLOADS[n] for n in CURVE_WORKLOADS]
+    assert [w.N for w in ws] == [128, 2048, 4096, 16384, 8192]
+    # the longest sequence (the curve's axis); C3, C4 and C5 hold equally many Q elements
+    assert max(ws, key=lambda w: w.N).name == DEFAULT_BENCH_WORKLOAD

@@ -68,3 +68,27 @@ def test_bench_line(case):
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     # a few samples at most in so short a run; the key is always present
     assert j["clocks"] is None or j["clocks"]["sm_mhz"] > 0
+
+
+def test_default_line_carries_the_curve():
+    """The default run times the largest forward configuration and adds
+    per_config: all five forward configurations, shortest sequence first,
+    each with its own value, roofline and probed SM clock."""
+    from exact_io_aware_78_b200.inputs import CURVE_WORKLOADS, DEFAULT_BENCH_WORKLOAD
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--steps", str(STEPS), "--warmup", "3",
+           "--no-cpu-baseline"]
+    proc = subprocess.run(cmd, capture_output=True, text=True, timeout=280, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    lines = [l for l in proc.stdout.splitlines() if l.lstrip().startswith("{")]
+    assert len(lines) == 1, proc.stdout
+    j = json.loads(lines[0])
+    assert j["config"]["workload"] == DEFAULT_BENCH_WORKLOAD
+    curve = j["per_config"]
+    assert [c["workload"] for c in curve] == list(CURVE_WORKLOADS)
+    for c in curve:
+        r = c["roofline"]
+        assert c["value"] > 0 and c["ms_per_step"] > 0 and r["achieved"] > 0
+        assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], rel=1e-9)
+        assert c["clocks"]["sm_mhz_probe_median"] > 100
+    top = curve[list(CURVE_WORKLOADS).index(DEFAULT_BENCH_WORKLOAD)]
+    assert top["value"] == j["value"] and top["roofline"] == j["roofline"]
