@@ -940,9 +940,10 @@ def spawn_ranks(gpus: int) -> int:
 def measure_peaks(args):
     """Dense matmul peaks on this GPU for the roofline denominators: torch
     bf16 matmul and e4m3 torch._scaled_mm (bf16 output, unit scales) at
-    8192^3, best of 10 back-to-back calls (burst) and the mean over about 4 s
-    of back-to-back calls (sustained, under the power cap), with the SM
-    clock sampled during each.  Prints one JSON line."""
+    8192^3.  Burst: best of 10 single calls, each followed by an SM clock
+    probe, taken for both formats (after a short idle, twice) before any
+    long load; sustained: back-to-back calls for about --peak-seconds each,
+    with nvidia-smi clocks sampled meanwhile.  Prints one JSON line."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     n = 8192
@@ -960,21 +961,30 @@ def measure_peaks(args):
              "fp8": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)}
     flop = 2.0 * n ** 3
     out = {"what": "dense matmul peaks, 8192^3", "gpu": torch.cuda.get_device_name(dev)}
-    for name, fn in kinds.items():
-        for _ in range(5):
-            fn()
-        torch.cuda.synchronize(dev)
-        best = float("inf")
-        mhz = []
-        for _ in range(10):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-            ev = sm_clock_probe(stream)
+    best = {k: float("inf") for k in kinds}
+    mhz = {k: [] for k in kinds}
+    for rnd in range(2):
+        for name, fn in kinds.items():
+            time.sleep(1.0)
+            for _ in range(3):
+                fn()
             torch.cuda.synchronize(dev)
-            best = min(best, e0.elapsed_time(e1))
-            mhz.append(probe_mhz(ev))
+            for _ in range(10):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                ev = sm_clock_probe(stream)
+                torch.cuda.synchronize(dev)
+                t = e0.elapsed_time(e1)
+                if t < best[name]:
+                    best[name] = t
+                mhz[name].append(probe_mhz(ev))
+    for name, fn in kinds.items():
+        out[f"{name}_tflops"] = flop / (best[name] * 1e-3) / 1e12
+        out[f"{name}_burst_sm_mhz_probe_median"] = statistics.median(mhz[name])
+    for name, fn in kinds.items():
+        time.sleep(2.0)
         sampler = ClockSampler(0)
         sampler.start()
         t_end = time.perf_counter() + args.peak_seconds
@@ -988,12 +998,10 @@ def measure_peaks(args):
             torch.cuda.synchronize(dev)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        clocks = sampler.stop()
-        out[f"{name}_tflops"] = flop / (best * 1e-3) / 1e12
         out[f"{name}_tflops_sustained"] = flop * calls / (e0.elapsed_time(e1) * 1e-3) / 1e12
-        out[f"{name}_burst_sm_mhz_probe_median"] = statistics.median(mhz)
-        out[f"{name}_sustained_clocks"] = clocks
+        out[f"{name}_sustained_clocks"] = sampler.stop()
     out["fp8_over_bf16_burst"] = out["fp8_tflops"] / out["bf16_tflops"]
+    out["fp8_over_bf16_sustained"] = out["fp8_tflops_sustained"] / out["bf16_tflops_sustained"]
     print(json.dumps(out), flush=True)
 
 

@@ -101,11 +101,11 @@ struct KernelCfg {
   static constexpr int BM = 128;          // query rows per tile
   static constexpr int BN = 128;          // keys per K/V tile
   static constexpr int kTiles = 2;        // query tiles per work item
-  // Warpgroups 0, 1: softmax of query tile 0, 1.  Warpgroup 2: warp 8 issues
-  // the MMAs, warp 9 issues the TMA copies, warps 10-11 only hold the
-  // warpgroup's register budget.  Launch budget 384 x 168 registers; the
-  // split below gives the softmax threads 216 and warpgroup 2 72:
-  // 256 * 216 + 128 * 72 = 64512 = 384 * 168.
+  // Warpgroups 0, 1: softmax and epilogue of query tile 0, 1.  Warpgroup 2:
+  // warp 8 issues the MMAs, warp 9 the TMA loads, warps 10-11 only hold the
+  // warpgroup's register budget.  Launch budget
+  // 384 x 168 registers; the split below gives the softmax threads 216 and
+  // warpgroup 2 72: 256 * 216 + 128 * 72 = 64512 = 384 * 168.
   static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = 168;
   static constexpr int kSoftmaxRegs = 216;
@@ -119,6 +119,7 @@ struct KernelCfg {
   static constexpr int kVBytes = kVChunks * kChunkBytes;
   static constexpr int kStageBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr int kKStep = 32 / kEsize;            // K extent of one MMA (32 bytes)
+  static constexpr int kOutEsize = kOut == kOutF32Split ? 4 : 2;  // bytes per O element
   static constexpr int kSmemMax = 232448;               // per-CTA opt-in limit on sm_100
   static constexpr int kBarBytes = 1024;
   static constexpr int kStagesFit = (kSmemMax - 1024 - kBarBytes - kTiles * kQBytes) / kStageBytes;
@@ -131,7 +132,11 @@ struct KernelCfg {
   static constexpr int kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t * 128); }
   __host__ __device__ static constexpr uint32_t o_col(int t) { return static_cast<uint32_t>(256 + t * kDv); }
-  static constexpr float kTau = kEsize == 2 ? 8.0f : 8.0f;  // lazy-rescale threshold (log2 units)
+  // Lazy-rescale threshold (log2 units): probabilities stay below 2^kTau.
+  // bf16 P keeps its relative precision at any magnitude and the fp32 sums
+  // have ample range, so 16 costs nothing and makes moves of the reference
+  // (each one a rescale of O) rare; e4m3 P saturates at 448, so 8.
+  static constexpr float kTau = kEsize == 2 ? 16.0f : 8.0f;
   static constexpr float kPShift = 0.0f;                    // P stored as 2^kPShift * p
 
   static_assert(kDqk * kEsize % 128 == 0 && kDv * kEsize % 128 == 0, "head dims must fill 128-byte rows");
@@ -550,6 +555,54 @@ __device__ __forceinline__ float max128(const float (&x)[128]) {
   return fmaxf(fmax3(c[0], c[1], c[2]), fmaxf(c[3], c[4]));
 }
 
+// One pair of probabilities p = 2^(s cs - m) (the argument as one paired
+// FMA), added to the paired row sums and packed into P words: bf16 pairs,
+// or e4m3 quads (the first pair of a quad waits in e_prev).  I is the pair
+// index in the row (a constant once the callers' loops are unrolled).
+template <class C>
+__device__ __forceinline__ void prob_pair(int I, const float (&x)[128], uint64_t cs2, uint64_t nr2,
+                                          uint64_t (&acc)[2], uint32_t (&pk)[16], float (&e_prev)[2]) {
+  const uint64_t y = f2_fma(f2_pack(x[2 * I], x[2 * I + 1]), cs2, nr2);
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  const float e0 = ex2_approx(y0);
+  const float e1 = ex2_approx(y1);
+  const uint64_t e01 = f2_pack(e0, e1);
+  acc[I & 1] = I < 2 ? e01 : f2_add(acc[I & 1], e01);
+  if (C::kEsize == 2) {
+    pk[I & 15] = pack_bf16x2(e0, e1);
+  } else if (I & 1) {
+    pk[(I & 15) >> 1] = pack_e4m3x4(e_prev[0], e_prev[1], e0, e1);
+  } else {
+    e_prev[0] = e0;
+    e_prev[1] = e1;
+  }
+}
+
+// Keys [32 Q, 32 Q + 32) of the row (16 pairs), their P words stored over
+// the first columns of S (already read).  With kMax the same loop takes the
+// row maximum of all 128 scores for the first two quarters (two chains of
+// three-input maxima, interleaved with the exponentials and off their
+// critical path).
+template <class C, int Q, bool kMax>
+__device__ __forceinline__ void prob_quarter(const float (&x)[128], uint64_t cs2, uint64_t nr2, uint64_t (&acc)[2],
+                                             float (&e_prev)[2], float& mA, float& mB, uint32_t tS) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int I = 16 * Q + k;
+    if (kMax) {
+      mA = fmax3(mA, x[2 * I], x[2 * I + 1]);
+      mB = fmax3(mB, x[64 + 2 * I], x[65 + 2 * I]);
+    }
+    prob_pair<C>(I, x, cs2, nr2, acc, pk, e_prev);
+  }
+  if constexpr (C::kEsize == 2)
+    tmem_st16(tS + 16 * Q, pk);
+  else
+    tmem_st8(tS + 8 * Q, pk);
+}
+
 template <class C, bool kRanges>
 __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t tmem, int warp, int lane) {
   const int quad = warp & 3;
@@ -569,7 +622,7 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
     if (kRanges && r.lo >= r.hi) {  // no row of this tile sees a key: O = 0, LSE = -inf
       if (qrow < p.N) {
         const size_t row_elem = ((static_cast<size_t>(wk.b) * p.N + qrow) * p.Hq + wk.h) * C::kDout;
-        constexpr int kVec = C::kDout * (C::kOut == kOutBf16 ? 2 : 4) / 16;
+        constexpr int kVec = C::kDout * C::kOutEsize / 16;
         uint4* dst = C::kOut == kOutBf16 ? reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row_elem)
                                          : reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.o) + row_elem);
 #pragma unroll 4
@@ -592,7 +645,10 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
       key_lo = max(key_lo, __ldg(p.key_lo + ix));
       key_hi = min(key_hi, __ldg(p.key_hi + ix));
     }
+    const uint64_t cs2 = f2_pack(cs, cs);
 
+    // m_used: the reference maximum of the row's probabilities (log2 units),
+    // moved only when a tile's maximum exceeds it by more than kTau.
     float m_used = -CUDART_INF_F;
     float l = 0.0f;
     for (int j = r.lo; j < r.hi; ++j) {
@@ -625,73 +681,60 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
         for (int c = 0; c < 128; ++c)
           if (c < vlo || c >= vhi) x[c] = -CUDART_INF_F;
       }
-      const float m_tile = max128(x) * cs;
+      // The row's first visible keys set the reference before any
+      // exponential.  Later tiles start their exponentials at once against
+      // the reference in use while the tile's maximum is taken alongside;
+      // only a maximum above the reference by more than kTau (rare once a
+      // row's first tiles are done) moves it -- l and O are rescaled and the
+      // first half is computed again, so the probabilities are exactly those
+      // of moving the reference first.
+      if (m_used == -CUDART_INF_F) m_used = max128(x) * cs;
 
-      // Lazy rescale: move the reference max only when the new tile's max
-      // exceeds it by more than kTau.
-      float alpha = 1.0f;
-      bool rescale_o = false;
-      if (m_tile > m_used + C::kTau) {
-        alpha = ex2_approx(m_used - m_tile);  // 0 when m_used is -inf
-        rescale_o = (j > r.lo) && (m_used != -CUDART_INF_F);
-        l *= alpha;
-        m_used = m_tile;
-      }
-      if (__any_sync(0xFFFFFFFFu, rescale_o)) {
-        const float f = rescale_o ? alpha : 1.0f;
+      uint64_t acc[2];
+      float e_prev[2];
 #pragma unroll 1
-        for (int cc = 0; cc < C::kDv; cc += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + cc, ov);
-          tmem_wait_ld();
+      for (;;) {
+        const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used) + C::kPShift;
+        const uint64_t nr2 = f2_pack(neg_ref, neg_ref);
+        float mA = -CUDART_INF_F, mB = -CUDART_INF_F;
+        prob_quarter<C, 0, true>(x, cs2, nr2, acc, e_prev, mA, mB, tS);
+        prob_quarter<C, 1, true>(x, cs2, nr2, acc, e_prev, mA, mB, tS);
+        const float m_tile = fmaxf(mA, mB) * cs;
+        const bool up = m_tile > m_used + C::kTau;  // false while m_used is -inf: m_tile is then -inf too
+        if (!__any_sync(0xFFFFFFFFu, up)) {
+          // publish P of keys 0..63: the first half of P V can start
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->p_half[t]);
+          // keys 64..127 against the same reference
+          prob_quarter<C, 2, false>(x, cs2, nr2, acc, e_prev, mA, mB, tS);
+          prob_quarter<C, 3, false>(x, cs2, nr2, acc, e_prev, mA, mB, tS);
+          break;
+        }
+        float alpha = 1.0f;
+        bool rescale_o = false;
+        if (up) {
+          alpha = ex2_approx(m_used - m_tile);
+          rescale_o = j > r.lo;  // O holds products of earlier tiles (all finished: S(j) follows them)
+          l *= alpha;
+          m_used = m_tile;
+        }
+        if (__any_sync(0xFFFFFFFFu, rescale_o)) {
+          const float f = rescale_o ? alpha : 1.0f;
+#pragma unroll 1
+          for (int cc = 0; cc < C::kDv; cc += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + cc, ov);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-          tmem_st32(tO + cc, ov);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+            tmem_st32(tO + cc, ov);
+          }
         }
       }
-
-      // p = 2^(s cs - m): the argument in pairs, exp2 per element, the row
-      // sum in four paired partial sums, P packed and written over S.
       {
-        const float neg_ref = -((m_used == -CUDART_INF_F) ? 0.0f : m_used) + C::kPShift;
-        const uint64_t cs2 = f2_pack(cs, cs);
-        const uint64_t nr2 = f2_pack(neg_ref, neg_ref);
-        uint64_t acc[4];
-        // Two halves of 64 columns; each half's P words are stored before the
-        // next half is computed, so at most 32 packed words are live.
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[PWords<C>::kN / 2];
-#pragma unroll
-          for (int ii = 0; ii < 32; ++ii) {
-            const int i = h * 32 + ii;
-            const uint64_t y = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), cs2, nr2);
-            float y0, y1;
-            f2_unpack(y, y0, y1);
-            const float e0 = ex2_approx(y0);
-            const float e1 = ex2_approx(y1);
-            const uint64_t e01 = f2_pack(e0, e1);
-            acc[i & 3] = i < 4 ? e01 : f2_add(acc[i & 3], e01);
-            if (C::kEsize == 2) {
-              pk[ii] = pack_bf16x2(e0, e1);
-            } else {
-              x[2 * i] = e0;  // e4m3 packs four at a time
-              x[2 * i + 1] = e1;
-              if (ii & 1) pk[ii >> 1] = pack_e4m3x4(x[2 * i - 2], x[2 * i - 1], e0, e1);
-            }
-          }
-          if (C::kEsize == 2)
-            tmem_st32(tS + 32 * h, pk);
-          else
-            tmem_st16(tS + 16 * h, pk);
-          if (h == 0) {  // publish P of keys 0..63: the first half of P V can start
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->p_half[t]);
-          }
-        }
-        const uint64_t s2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        const uint64_t s2 = f2_add(acc[0], acc[1]);
         float s0, s1;
         f2_unpack(s2, s0, s1);
         l += s0 + s1;
@@ -702,58 +745,48 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
       if (lane == 0) mbar_arrive(&ctl->p_full[t]);
     }
 
-    // Epilogue: O = acc / l, LSE = ln 2 * (m + log2 l).
+    // Epilogue: O = acc / l, LSE = ln 2 * (m + log2 l).  The row of O is read
+    // from tensor memory at once and its columns are released before the
+    // stores, so the next item's first P V can start meanwhile.
     {
       bool ok = wait_phase(&ctl->o_full[t], o_phase, ctl, p, kSiteSoftOFull, true);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) return;
       o_phase ^= 1u;
       tc_fence_after();
-      const float inv_l = l > 0.0f ? out_mult / l : 0.0f;
-      const bool store = qrow < p.N;
-      const size_t row_elem = ((static_cast<size_t>(wk.b) * p.N + qrow) * p.Hq + wk.h) * C::kDout;
-      if (C::kOut == kOutBf16) {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row_elem);
-#pragma unroll 1
-        for (int cc = 0; cc < C::kDv; cc += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + cc, ov);
-          tmem_wait_ld();
-          uint32_t pk[16];
+      uint32_t ov[C::kDv];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
-          if (store) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[cc / 8 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row_elem);
-#pragma unroll 1
-        for (int cc = 0; cc < C::kDout; cc += 32) {
-          uint32_t hi_part[32], lo_part[32];
-          tmem_ld32(tO + cc, hi_part);
-          tmem_ld32(tO + C::kDout + cc, lo_part);
-          tmem_wait_ld();
-          if (store) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 v;
-              v.x = (__uint_as_float(hi_part[4 * i + 0]) + __uint_as_float(lo_part[4 * i + 0])) * inv_l;
-              v.y = (__uint_as_float(hi_part[4 * i + 1]) + __uint_as_float(lo_part[4 * i + 1])) * inv_l;
-              v.z = (__uint_as_float(hi_part[4 * i + 2]) + __uint_as_float(lo_part[4 * i + 2])) * inv_l;
-              v.w = (__uint_as_float(hi_part[4 * i + 3]) + __uint_as_float(lo_part[4 * i + 3])) * inv_l;
-              dst[cc / 4 + i] = v;
-            }
-          }
-        }
-      }
+      for (int cc = 0; cc < C::kDv; cc += 32) tmem_ld32p(tO + cc, ov + cc);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->o_empty[t]);
-      if (store) {
+      const float inv_l = l > 0.0f ? out_mult / l : 0.0f;
+      if (qrow < p.N) {
+        const size_t row_elem = ((static_cast<size_t>(wk.b) * p.N + qrow) * p.Hq + wk.h) * C::kDout;
+        if constexpr (C::kOut == kOutBf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row_elem);
+#pragma unroll
+          for (int g = 0; g < C::kDv / 8; ++g) {  // 8 bf16 columns per 16-byte store
+            const int c = g * 8;
+            dst[g] = make_uint4(pack_bf16x2(__uint_as_float(ov[c + 0]) * inv_l, __uint_as_float(ov[c + 1]) * inv_l),
+                                pack_bf16x2(__uint_as_float(ov[c + 2]) * inv_l, __uint_as_float(ov[c + 3]) * inv_l),
+                                pack_bf16x2(__uint_as_float(ov[c + 4]) * inv_l, __uint_as_float(ov[c + 5]) * inv_l),
+                                pack_bf16x2(__uint_as_float(ov[c + 6]) * inv_l, __uint_as_float(ov[c + 7]) * inv_l));
+          }
+        } else {  // fp32: the high and low halves of P V' summed, 4 columns per 16-byte store
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row_elem);
+#pragma unroll
+          for (int g = 0; g < C::kDout / 4; ++g) {
+            const int c = g * 4;
+            float4 v;
+            v.x = (__uint_as_float(ov[c + 0]) + __uint_as_float(ov[C::kDout + c + 0])) * inv_l;
+            v.y = (__uint_as_float(ov[c + 1]) + __uint_as_float(ov[C::kDout + c + 1])) * inv_l;
+            v.z = (__uint_as_float(ov[c + 2]) + __uint_as_float(ov[C::kDout + c + 2])) * inv_l;
+            v.w = (__uint_as_float(ov[c + 3]) + __uint_as_float(ov[C::kDout + c + 3])) * inv_l;
+            dst[g] = v;
+          }
+        }
         const float lse = l > 0.0f ? (m_used + __log2f(l) - C::kPShift) * 0.69314718055994531f
                                    : -CUDART_INF_F;
         p.lse[(static_cast<size_t>(wk.b) * p.Hq + wk.h) * p.N + qrow] = lse;

@@ -93,12 +93,6 @@ struct DecodeTcCfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-// Make this thread's ordinary shared-memory stores visible to the async
-// proxy (the tensor core reads the query tile through it).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 struct DecodeTcCtl {
   uint64_t full[8], empty[8];
   uint64_t q_full, q_empty;

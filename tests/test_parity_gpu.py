@@ -69,6 +69,61 @@ def test_sharpened_queries_stress_rescale():
     case(1, 2, 2, 512, 128, False, 0, "bf16", seed=78, q_mult=4.0)
 
 
+def _ramp_inputs(B, H, N, d, dtype, seed, ramp):
+    """Q = N(0, 1) + 1 and K[j] = N(0, 1) / 2 + ramp * j / N (every
+    dimension), V = N(0, 1): each row's scores grow along the keys, so its
+    running maximum climbs tile after tile."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, N, H, d, generator=g) + 1.0
+    k = torch.randn(B, N, H, d, generator=g) * 0.5 + (ramp * torch.arange(N) / N).view(1, N, 1, 1)
+    v = torch.randn(B, N, H, d, generator=g)
+    out = {"q_scale": None, "k_scale": None, "v_scale": None}
+    if dtype == "bf16":
+        out.update(q=q.bfloat16(), k=k.bfloat16(), v=v.bfloat16())
+    else:
+        from exact_io_aware_78_b200.inputs import quantize_e4m3_per_head
+        for n, x in (("q", q), ("k", k), ("v", v)):
+            out[n], out[n + "_scale"] = quantize_e4m3_per_head(x)
+    return out
+
+
+def _reference_moves(q, k, causal, scale, tau):
+    """How often each row's reference maximum must move under the kernel's
+    rule (set by the row's first visible 128-key tile, moved when a later
+    tile's maximum exceeds it by more than tau, in log2 units)."""
+    cs = scale / np.log(2.0)
+    s = np.einsum("bihd,bjhd->bhij", q, k) * cs
+    N = s.shape[-1]
+    if causal:
+        s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+    tm = np.stack([s[..., j:j + 128].max(-1) for j in range(0, N, 128)], -1)
+    ref = tm[..., 0].copy()
+    moves = np.zeros(ref.shape, int)
+    for t in range(1, tm.shape[-1]):
+        up = tm[..., t] > ref + tau
+        moves += up
+        ref = np.where(up, tm[..., t], ref)
+    return moves
+
+
+@pytest.mark.parametrize("dtype,tau", [("bf16", 16.0), ("fp8", 8.0)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_growing_scores_move_the_reference(dtype, tau, causal):
+    """Scores that grow along the keys make every row's reference maximum
+    move several times, so the rescale of l and O (and, for the first half of
+    a tile computed against the old reference, its recomputation) runs on
+    most steps; the result must still match the oracle."""
+    B, H, N, d = 1, 2, 1000, 128
+    inp = _ramp_inputs(B, H, N, d, dtype, 4040 + causal, ramp=8.0)
+    q, k, v = oracle_view(inp, dtype)
+    moves = _reference_moves(q, k, causal, d ** -0.5, tau)
+    rows_seen = moves[..., 256:]  # rows that see at least three tiles
+    assert np.median(rows_seen) >= 2, "inputs do not exercise the rescale path"
+    O, L = run_gpu(inp, causal, 0, d ** -0.5)
+    Oref, Lref = attention_ref(q, k, v, causal, 0, d ** -0.5)
+    assert_close(O, L, Oref, Lref, dtype, f"growing scores {dtype} causal={causal}")
+
+
 # --------------------------------------------------------- full workloads
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_workload_sampled_rows(name):
