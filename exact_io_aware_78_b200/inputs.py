@@ -138,6 +138,30 @@ def make_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, dtype: str, seed: int
     return out
 
 
+def make_ramp_inputs(B: int, H: int, N: int, d: int, dtype: str, seed: int,
+                     ramp: float) -> Dict[str, Optional[torch.Tensor]]:
+    """Inputs whose scores grow along the keys: Q = N(0, 1) + 1 and
+    K[j] = N(0, 1) / 2 + ramp * j / N in every dimension, V = N(0, 1) (one
+    generator seeded with `seed`, drawn in that order), stored bf16 or as
+    e4m3 codes with per-head scales.  Each row's running maximum then climbs
+    from key tile to key tile, which exercises the rescaling of the running
+    sums."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn(B, N, H, d, generator=g) + 1.0
+    k = torch.randn(B, N, H, d, generator=g) * 0.5 + (ramp * torch.arange(N) / N).view(1, N, 1, 1)
+    v = torch.randn(B, N, H, d, generator=g)
+    out: Dict[str, Optional[torch.Tensor]] = {"q_scale": None, "k_scale": None, "v_scale": None}
+    if dtype == "bf16":
+        out.update(q=q.to(torch.bfloat16), k=k.to(torch.bfloat16), v=v.to(torch.bfloat16))
+    elif dtype == "fp8":
+        for name, x in (("q", q), ("k", k), ("v", v)):
+            out[name], out[name + "_scale"] = quantize_e4m3_per_head(x)
+    else:
+        raise ValueError(f"unknown dtype {dtype!r}")
+    return out
+
+
 def workload_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
     out = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.seed, w.q_mult)
     out["key_lo"] = out["key_hi"] = None

@@ -6,7 +6,7 @@ import torch
 
 import exact_io_aware_78_b200 as ea
 from exact_io_aware_78_b200 import _binding as Bn
-from exact_io_aware_78_b200.inputs import WORKLOADS, make_inputs, sample_rows, workload_inputs
+from exact_io_aware_78_b200.inputs import WORKLOADS, make_inputs, make_ramp_inputs, sample_rows, workload_inputs
 from oracle import attention_ref
 
 from gpu_helpers import assert_close, case, oracle_view, ranges_view, run_gpu
@@ -69,24 +69,6 @@ def test_sharpened_queries_stress_rescale():
     case(1, 2, 2, 512, 128, False, 0, "bf16", seed=78, q_mult=4.0)
 
 
-def _ramp_inputs(B, H, N, d, dtype, seed, ramp):
-    """Q = N(0, 1) + 1 and K[j] = N(0, 1) / 2 + ramp * j / N (every
-    dimension), V = N(0, 1): each row's scores grow along the keys, so its
-    running maximum climbs tile after tile."""
-    g = torch.Generator().manual_seed(seed)
-    q = torch.randn(B, N, H, d, generator=g) + 1.0
-    k = torch.randn(B, N, H, d, generator=g) * 0.5 + (ramp * torch.arange(N) / N).view(1, N, 1, 1)
-    v = torch.randn(B, N, H, d, generator=g)
-    out = {"q_scale": None, "k_scale": None, "v_scale": None}
-    if dtype == "bf16":
-        out.update(q=q.bfloat16(), k=k.bfloat16(), v=v.bfloat16())
-    else:
-        from exact_io_aware_78_b200.inputs import quantize_e4m3_per_head
-        for n, x in (("q", q), ("k", k), ("v", v)):
-            out[n], out[n + "_scale"] = quantize_e4m3_per_head(x)
-    return out
-
-
 def _reference_moves(q, k, causal, scale, tau):
     """How often each row's reference maximum must move under the kernel's
     rule (set by the row's first visible 128-key tile, moved when a later
@@ -114,7 +96,7 @@ def test_growing_scores_move_the_reference(dtype, tau, causal):
     a tile computed against the old reference, its recomputation) runs on
     most steps; the result must still match the oracle."""
     B, H, N, d = 1, 2, 1000, 128
-    inp = _ramp_inputs(B, H, N, d, dtype, 4040 + causal, ramp=8.0)
+    inp = make_ramp_inputs(B, H, N, d, dtype, 4040 + causal, ramp=8.0)
     q, k, v = oracle_view(inp, dtype)
     moves = _reference_moves(q, k, causal, d ** -0.5, tau)
     rows_seen = moves[..., 256:]  # rows that see at least three tiles
