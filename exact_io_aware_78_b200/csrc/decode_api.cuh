@@ -8,6 +8,26 @@
 // decode_tc_kernel.cuh over a stream-K split of all K/V tiles; with an
 // explicit split count the CUDA-core kernel of decode_kernel.cuh.
 
+// The combine kernel, launched as a programmatic dependent of the key-range
+// kernel queued just before it: its blocks may be scheduled while that
+// kernel finishes, and wait in-kernel for its completion before reading the
+// partials, so the launch gap between the two disappears.
+static int launch_combine(int d, unsigned blocks, const ea::DecodeParams& cp, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(32 * ea::kDecodeWarps);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = d == 128 ? cudaLaunchKernelEx(&cfg, ea::decode_combine_kernel<128>, cp)
+                                 : cudaLaunchKernelEx(&cfg, ea::decode_combine_kernel<64>, cp);
+  return e == cudaSuccess ? EA_OK : EA_ELAUNCH;
+}
+
 // Tensor map over q [B, Nq, Hq, d] with boxes of 128 bytes x `group` heads x
 // Nq rows: one box is the query rows of one key/value head's group.
 static int make_group_q_map(CUtensorMap* m, const void* base, int d, int Hq, int Nq, int B, int group) {
@@ -97,13 +117,7 @@ static int decode_tc_launch(const void* q, const void* k, const void* v, void* o
   if (rc == EA_OK) {
     kern<<<static_cast<unsigned>(G), 192, smem, stream>>>(tq, tk, tv, tp);
     const unsigned comb_blocks = static_cast<unsigned>((pairs * rows + ea::kDecodeWarps - 1) / ea::kDecodeWarps);
-    if (cudaGetLastError() == cudaSuccess) {
-      if (d == 128)
-        ea::decode_combine_kernel<128><<<comb_blocks, 32 * ea::kDecodeWarps, 0, stream>>>(cp);
-      else
-        ea::decode_combine_kernel<64><<<comb_blocks, 32 * ea::kDecodeWarps, 0, stream>>>(cp);
-    }
-    rc = cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
+    rc = cudaGetLastError() == cudaSuccess ? launch_combine(d, comb_blocks, cp, stream) : EA_ELAUNCH;
   }
   cudaFreeAsync(scratch, stream);
   return rc;
@@ -199,13 +213,7 @@ int attn_fwd_decode(const void* q, const void* k, const void* v, void* o, float*
   const unsigned comb_blocks =
       static_cast<unsigned>((static_cast<long long>(B) * Hkv * rows + ea::kDecodeWarps - 1) / ea::kDecodeWarps);
   split<<<split_blocks, 32 * ea::kDecodeWarps, smem, stream>>>(p);
-  if (cudaGetLastError() == cudaSuccess) {
-    if (d == 128)
-      ea::decode_combine_kernel<128><<<comb_blocks, 32 * ea::kDecodeWarps, 0, stream>>>(p);
-    else
-      ea::decode_combine_kernel<64><<<comb_blocks, 32 * ea::kDecodeWarps, 0, stream>>>(p);
-  }
-  rc = cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
+  rc = cudaGetLastError() == cudaSuccess ? launch_combine(d, comb_blocks, p, stream) : EA_ELAUNCH;
   cudaFreeAsync(scratch, stream);
   return rc;
 }

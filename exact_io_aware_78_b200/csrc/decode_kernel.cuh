@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
   // shared memory: per warp the staged query rows [kRows][kD] (fp32, scaled)
   // and the batch's probabilities [32 keys][kRows]
   extern __shared__ float dec_smem[];
+  launch_dependents();  // the combine kernel may be scheduled; it waits for this grid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long task = static_cast<long long>(blockIdx.x) * kDecodeWarps + warp;
   const long long tasks = static_cast<long long>(p.B) * p.Hkv * p.splits;
@@ -298,6 +299,9 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_combine_kernel(const
   const int b = bk / p.Hkv, hkv = bk - b * p.Hkv;
   const int hg = r / p.Nq, i = r - hg * p.Nq;
   const int h = hkv * p.group + hg;
+  // The partials come from the key-range kernel queued just before this one
+  // (a programmatic dependent launch: this grid may start early).
+  grid_dependency_wait();
 
   // Ranges' weights computed across lanes (lane t handles ranges t, t + 32,
   // ...): M = max m over ranges with l > 0, then w = 2^(m - M) (0 for an

@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   DecodeTcCtl* ctl = reinterpret_cast<DecodeTcCtl*>(smem + G::kCtlOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  launch_dependents();  // the combine kernel may be scheduled; it waits for this grid
   // Rows R..127 of the query tile stay zero (the box fills rows 0..R-1).
   for (int i = threadIdx.x; i < G::kTileBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + G::kQOffset)[i] = make_uint4(0, 0, 0, 0);

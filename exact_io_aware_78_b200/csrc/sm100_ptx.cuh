@@ -412,6 +412,18 @@ __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// --------------------------------------------- programmatic dependent launch
+// Let the grid queued after this one on the stream (launched with
+// programmatic stream serialization) be scheduled now; it still waits in
+// grid_dependency_wait for this grid's completion.
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grid this one depends on has completed and its memory
+// operations are visible (a no-op when launched without the dependency).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
