@@ -10,11 +10,13 @@ from exact_io_aware_78_b200.inputs import make_inputs
 from oracle import attention_ref, dequantize_per_head
 
 # Correctness bars: max |O - O_ref|, mean |O - O_ref|, max |LSE - LSE_ref|.
-# bf16 and fp32 inputs: 2e-2 / 2e-3 / 1e-3.  e4m3 inputs: max 6e-2; the mean
-# bar 1e-2 and LSE bar 1e-3 are derived (P enters the second product as e4m3,
-# relative step 2^-4, so per-row errors average to a few 1e-3; LSE uses fp32
-# sums of unquantised probabilities).
-TOL = {"bf16": (2e-2, 2e-3, 1e-3), "fp32": (2e-2, 2e-3, 1e-3), "fp8": (6e-2, 1e-2, 1e-3)}
+# bf16 and fp32 inputs: 2e-2 / 2e-3 / 1e-3 (the stated bars).  e4m3 inputs:
+# max 6e-2 (stated); the mean bar 9e-3 is about twice the largest mean error
+# measured on a B200 over every e4m3 case (4.5e-3, on scores that grow along
+# the keys; P enters the second product as e4m3, relative step 2^-4, so
+# per-row errors average to a few 1e-3) and the LSE bar 1e-3 is the bf16 one
+# (LSE uses fp32 sums of unquantised probabilities).
+TOL = {"bf16": (2e-2, 2e-3, 1e-3), "fp32": (2e-2, 2e-3, 1e-3), "fp8": (6e-2, 9e-3, 1e-3)}
 
 
 def oracle_view(inp, dtype):

@@ -18,12 +18,15 @@ from oracle import attention_bwd_ref, attention_ref
 
 pytestmark = pytest.mark.gpu
 
-# Bars, relative to the size of each reference gradient: max |err| <= 2e-2 *
-# max |ref| and mean |err| <= 1e-2 * mean |ref|.  The kernels round P and dS
-# to bf16 (relative step 2^-9) before the products that consume them and
-# store bf16 gradients, and accumulate in fp32, so each gradient element
-# carries errors of a few 2^-9 of the typical element size.
-TOL_MAX, TOL_MEAN = 2e-2, 1e-2
+# Bars, relative to the size of each reference gradient: max |err| <= 1.2e-2
+# * max |ref| and mean |err| <= 6e-3 * mean |ref|, about twice the largest
+# errors measured on a B200 over every case in this file (relative max
+# 6.0e-3, relative mean 3.1e-3).  The kernels round P and dS to bf16
+# (relative step 2^-9) before the products that consume them and store bf16
+# gradients, accumulating in fp32, so each gradient element carries errors
+# of a few 2^-9 of the typical element size; a dropped term or a wrong
+# scale moves the mean by far more.
+TOL_MAX, TOL_MEAN = 1.2e-2, 6e-3
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -4,10 +4,11 @@ owns the device memory, or a runtime that needs a footprint fixed at load
 time).  It keeps its split operands in the library's static device array
 instead of allocating scratch on each call.
 
-Checked through the C ABI against the existing attn_fwd fp32 path, within
-the tolerances the other parity tests use, on two calls in a row (the second
-with other shapes and values, so stale contents of the shared array would
-show).  This file is collected last on purpose."""
+Checked through the C ABI against the existing attn_fwd fp32 path and
+against the float64 oracle, within the tolerances the other parity tests
+use, on two calls in a row (the second with other shapes and values, so
+stale contents of the shared array would show).  This file is collected last
+on purpose."""
 import pytest
 import torch
 
@@ -15,7 +16,9 @@ import exact_io_aware_78_b200 as ea
 from exact_io_aware_78_b200 import _binding as Bn
 from exact_io_aware_78_b200.inputs import make_inputs
 
-from gpu_helpers import TOL
+from oracle import attention_ref
+
+from gpu_helpers import TOL, assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -96,6 +99,25 @@ def test_noalloc_matches_attn_fwd_on_two_calls_in_a_row(lib):
     assert torch.cuda.mem_get_info(0)[0] == free_before
     for (o, lse), ref in zip(results, refs + [refs[0]]):
         _compare(o, lse, ref[5], ref[6])
+        q, k, v, causal, window = (x.double().cpu().numpy() if torch.is_tensor(x) else x for x in ref[:5])
+        Oref, Lref = attention_ref(q, k, v, causal, window, q.shape[-1] ** -0.5)
+        assert_close(o.double().cpu().numpy(), lse.double().cpu().numpy(), Oref, Lref, "fp32", "no-alloc vs oracle")
+
+
+def test_noalloc_set_up_again_after_shutdown(lib):
+    """attn_shutdown ends the per-device set-up: the next call looks the
+    array's address up again (and stays correct)."""
+    dev = torch.device("cuda:0")
+    inp = make_inputs(1, 2, 1, 200, 64, "fp32", 99)
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    rc, o1, l1 = _noalloc(lib, q, k, v, True, 0, None)
+    assert rc == Bn.EA_OK
+    torch.cuda.synchronize()
+    assert lib.attn_shutdown() == Bn.EA_OK
+    rc, o2, l2 = _noalloc(lib, q, k, v, True, 0, None)
+    assert rc == Bn.EA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
 def test_noalloc_rejects_requests_above_the_static_scratch(lib):
