@@ -405,17 +405,6 @@ __device__ __forceinline__ void mma_qk(uint32_t d_s, uint32_t q_lo, uint32_t k_l
   }
 }
 
-// A barrier test taken ahead of time (peek) and the wait it stands for
-// (settle): the warp goes on at once when every lane's peek saw the phase
-// complete, and otherwise falls back to the bounded wait.
-__device__ __forceinline__ bool peek(uint64_t* bar, uint32_t parity) { return mbar_test_wait(smem_u32(bar), parity); }
-
-__device__ __forceinline__ bool settle(bool peeked, uint64_t* bar, uint32_t parity, SharedCtl* ctl, const FwdParams& p,
-                                       int site) {
-  if (__all_sync(0xFFFFFFFFu, peeked)) return true;
-  return warp_wait_phase(bar, parity, ctl, p, site, true);
-}
-
 // The MMA issuer.  Per K/V step j of a work item it issues, in order:
 //   O_0 += P_0(j-1) V(j-1)  in two halves (keys 0-63 once the softmax has
 //                           published them, then keys 64-127),
@@ -424,11 +413,13 @@ __device__ __forceinline__ bool settle(bool peeked, uint64_t* bar, uint32_t pari
 //   S_1 = Q_1 K(j)^T,                         then releases K(j).
 // S_T(j) overwrites the columns that held P_T(j-1), so it must follow
 // O_T += P_T(j-1) V(j-1) (the tensor core runs one thread's MMAs in order).
-// Every barrier the issuer needs is tested one MMA batch before it is
-// needed, so that the test's latency hides behind the MMA issue.  Waits on
-// the softmax's P and on O being free (tensor memory written or read by
-// other threads) are followed by tcgen05.fence::after_thread_sync; waits on
-// copies into shared memory need none.
+// An mbarrier test costs the warp about 150 cycles even when the phase is
+// complete, so none sits between a tile's P and its next S: both ring
+// stages of the step (V(j-1), K(j)), which land well ahead, are checked at
+// the start of the step, and each P is waited for right before its
+// product.  Waits on P and on O being free (tensor memory written or read
+// by other threads) are followed by tcgen05.fence::after_thread_sync; waits
+// on copies into shared memory need none.
 template <class C, bool kRanges>
 __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint32_t tmem) {
   constexpr uint32_t kStageUnits = C::kStageBytes >> 4;
@@ -467,56 +458,44 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
       q_phase[1] ^= 1u;
     }
     if (!ok) break;
-    bool pk_v = false, pk_half0 = false;  // peeked during the previous step
     for (int j = lo; j <= hi; ++j) {
+      // The step's ring stages: V(j-1), then K(j).
       uint32_t v_stage = 0, k_stage = 0;
-      if (j > lo) {  // V(j-1) is next in ring order
-        ok = settle(pk_v, &ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull);
+      if (j > lo) {
+        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
         if (!ok) break;
         v_stage = cur.stage;
         cur.advance();
       }
+      if (j < hi) {
+        ok = warp_wait_phase(&ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull, true);
+        if (!ok) break;
+        k_stage = cur.stage;
+        cur.advance();
+      }
       const uint32_t v_lo = v_lo_base + v_stage * kStageUnits;
-      bool pk_k = false, pk_half1 = false;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const TileRange& rt = r[t];
         if (rt.active && j - 1 >= rt.lo && j - 1 < rt.hi) {  // O_t += P_t(j-1) V(j-1)
           const uint32_t d_o = tmem + C::o_col(t);
           const uint32_t a_p = tmem + C::s_col(t);
-          ok = settle(t == 0 ? pk_half0 : pk_half1, &ctl->p_half[t], p_phase[t], ctl, p, kSiteMmaPFull);
+          ok = warp_wait_phase(&ctl->p_half[t], p_phase[t], ctl, p, kSiteMmaPFull, true);
           if (ok && j - 1 == rt.lo) {  // first product of this item: the previous epilogue must be done with O_t
             ok = warp_wait_phase(&ctl->o_empty[t], (o_iter[t] & 1u) ^ 1u, ctl, p, kSiteMmaOEmpty, true);
             ++o_iter[t];
           }
           if (!ok) break;
           tc_fence_after();
-          const bool pk_full = peek(&ctl->p_full[t], p_phase[t]);
           mma_pv<C, 0, kHalf>(d_o, a_p, v_lo, kIdO, (j - 1 > rt.lo) ? 1u : 0u);
-          ok = settle(pk_full, &ctl->p_full[t], p_phase[t], ctl, p, kSiteMmaPFull);
+          ok = warp_wait_phase(&ctl->p_full[t], p_phase[t], ctl, p, kSiteMmaPFull, true);
           if (!ok) break;
           p_phase[t] ^= 1u;
           tc_fence_after();
-          if (t == 0 && j < hi) pk_k = peek(&ctl->full[cur.stage], cur.phase);
           mma_pv<C, kHalf, 2 * kHalf>(d_o, a_p, v_lo, kIdO, 1u);
           if (j - 1 == rt.hi - 1) mma_commit_elect(&ctl->o_full[t]);
         }
-        if (t == 0) {
-          if (j < hi) {  // K(j)
-            ok = settle(pk_k, &ctl->full[cur.stage], cur.phase, ctl, p, kSiteMmaKvFull);
-            if (!ok) break;
-            k_stage = cur.stage;
-            cur.advance();
-          }
-          if (r[1].active && j - 1 >= r[1].lo && j - 1 < r[1].hi) pk_half1 = peek(&ctl->p_half[1], p_phase[1]);
-        } else if (j > lo) {
-          mma_commit_elect(&ctl->empty[v_stage]);
-          // for the next step: V(j), next in ring order, and P_0(j)
-          if (j < hi) {
-            pk_v = peek(&ctl->full[cur.stage], cur.phase);
-            if (r[0].active && j >= r[0].lo && j < r[0].hi) pk_half0 = peek(&ctl->p_half[0], p_phase[0]);
-          }
-        }
+        if (t == 1 && j > lo) mma_commit_elect(&ctl->empty[v_stage]);
         if (rt.active && j >= rt.lo && j < rt.hi) {  // S_t = Q_t K(j)^T
           mma_qk<C, 0>(tmem + C::s_col(t), q_lo[t], k_lo_base + k_stage * kStageUnits, kIdS);
           mma_commit_elect(&ctl->s_full[t]);
