@@ -20,6 +20,7 @@ EA_BF16, EA_FP8_E4M3, EA_FP32 = 0, 1, 2
 EA_OK, EA_EINVAL, EA_EUNSUPPORTED, EA_EALIGN, EA_ELAUNCH, EA_EDEVICE_TIMEOUT, EA_ECUDA, EA_ENOMEM = (
     0, -1, -2, -3, -4, -5, -6, -7)
 EA_OPT_WAIT_TIMEOUT_NS, EA_OPT_MAX_CTAS, EA_OPT_SCHEDULE_ORDER, EA_OPT_SKIP_ARRIVE_ONCE = 1, 2, 3, 4
+EA_OPT_ITEM_DEAL = 5
 
 # Every function the header declares, with its ctypes signature.
 _SIGNATURES = {

@@ -9,7 +9,10 @@
 //   * One persistent CTA per SM walks work items (batch b, query head h,
 //     256-row query block) in a static heaviest-first order: parallelism over
 //     sequence blocks of one head ("FlashAttention-2 (PL)", "Ulepszony
-//     rownoleglosc").
+//     rownoleglosc").  With per-row key ranges, whose costs follow no order,
+//     each CTA instead takes its next item from a global counter when it
+//     starts one (a dynamic deal), and its load warp hands the item to the
+//     other roles.
 //   * A work item holds two 128-row query tiles of the same (b, h).  They
 //     share every K/V tile the TMA warp streams through a shared-memory ring,
 //     and ping-pong on the tensor core: while one tile's softmax runs on the
@@ -60,7 +63,9 @@ enum : int {
   kSiteSoftSFull = 7,
   kSiteSoftOFull = 8,
   kSiteMmaDrain = 9,
-  kSiteProdDrain = 10
+  kSiteProdDrain = 10,
+  kSiteItemFull = 11,   // row ranges: a consumer waiting for the next work item
+  kSiteItemEmpty = 12   // row ranges: the load warp waiting for a free item slot
 };
 
 // Output modes of the epilogue.
@@ -80,6 +85,8 @@ struct FwdParams {
   const int* key_hi;     // [B, N]
   const int2* tile_kv;   // [B, num_qtiles] K/V tile range [x, y) of each 128-row query tile (with ranges)
   const int* item_order; // [B * num_qblk] (batch, query block) pairs, most K/V tiles first (with ranges), or null
+  int* item_counter;     // with ranges: the dynamic deal's counter of items taken after each CTA's first
+                         // (zeroed before the launch), or null for the static deal
   int num_qtiles;        // ceil(N / 128)
   int B, Hq, Hkv, N, group;
   int causal, window;
@@ -160,6 +167,9 @@ struct SharedCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  uint64_t item_full[2];   // row ranges: the load warp has published work item item[s]
+  uint64_t item_empty[2];  // every consumer has read item[s]
+  int4 item[2];            // (b, h, hkv, qblk); qblk < 0: no more items
 };
 static_assert(sizeof(SharedCtl) <= 1024, "control block");
 
@@ -290,6 +300,52 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, 
   return __all_sync(0xFFFFFFFFu, wait_phase(bar, parity, ctl, p, site, honor_abort));
 }
 
+// ------------------------------------------------- work items (row ranges)
+// The kernel with per-row key ranges hands work items from the load warp to
+// the MMA warp and the eight softmax warps through two shared-memory slots:
+// the load warp ranks and decodes the CTA's i-th item and publishes it in
+// slot i % 2.  With a counter the item is the CTA's own block index first,
+// then gridDim.x plus the counter's next value (a dynamic deal: a CTA takes
+// more work when it is free, so unequal item costs still fill every SM);
+// without one, the static deal's rank.  A rank >= num_work publishes
+// qblk = -1 and ends every role's walk.  (The causal / window kernel, whose
+// static deal balances, computes its items in every role and has no slots.)
+template <bool kRanges>
+__device__ __forceinline__ bool publish_item(int i, WorkItem& wk, const FwdParams& p, SharedCtl* ctl) {
+  const int w = p.item_counter == nullptr ? work_rank(i)
+                : i == 0                  ? static_cast<int>(blockIdx.x)
+                                          : static_cast<int>(gridDim.x) + atomicAdd(p.item_counter, 1);
+  if (w < p.num_work) {
+    wk = decode_work<kRanges>(w, p);
+  } else {
+    wk.b = wk.h = wk.hkv = 0;
+    wk.qblk = -1;
+  }
+  const int s = i & 1;
+  if (!wait_phase(&ctl->item_empty[s], ((static_cast<uint32_t>(i) >> 1) & 1u) ^ 1u, ctl, p, kSiteItemEmpty, true))
+    return false;
+  ctl->item[s] = make_int4(wk.b, wk.h, wk.hkv, wk.qblk);  // ordered before the arrive by its memory clobber
+  mbar_arrive(&ctl->item_full[s]);
+  return true;
+}
+
+// Every lane of a consumer warp calls this; lane 0 frees the slot once the
+// whole warp has read it.
+__device__ __forceinline__ bool take_item(int i, WorkItem& wk, const FwdParams& p, SharedCtl* ctl, int lane) {
+  const int s = i & 1;
+  const bool ok = __all_sync(0xFFFFFFFFu, wait_phase(&ctl->item_full[s], (static_cast<uint32_t>(i) >> 1) & 1u, ctl,
+                                                     p, kSiteItemFull, true));
+  if (!ok) return false;
+  const int4 v = ctl->item[s];  // read after the wait (its asm has a memory clobber)
+  wk.b = v.x;
+  wk.h = v.y;
+  wk.hkv = v.z;
+  wk.qblk = v.w;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&ctl->item_empty[s]);
+  return true;
+}
+
 // ------------------------------------------------------------- TMA producer
 template <class C, bool kRanges>
 __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
@@ -303,9 +359,15 @@ __device__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
   uint32_t skipped_pos = 0xFFFFFFFFu;
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
-    if (w >= p.num_work) break;
-    const WorkItem wk = decode_work<kRanges>(w, p);
+    WorkItem wk;
+    if constexpr (kRanges) {
+      ok = publish_item<kRanges>(i, wk, p, ctl);
+      if (!ok || wk.qblk < 0) break;
+    } else {
+      const int w = work_rank(i);
+      if (w >= p.num_work) break;
+      wk = decode_work<kRanges>(w, p);
+    }
     const TileRange r0 = tile_range<kRanges>(wk, 0, p);
     const TileRange r1 = tile_range<kRanges>(wk, 1, p);
     int lo, hi;  // K/V tiles of the item: the span of both tiles' ranges
@@ -435,9 +497,15 @@ __device__ void mma_role(const FwdParams& p, SharedCtl* ctl, uint8_t* smem, uint
   uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, o_iter[2] = {0, 0};
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
-    if (w >= p.num_work) break;
-    const WorkItem wk = decode_work<kRanges>(w, p);
+    WorkItem wk;
+    if constexpr (kRanges) {
+      ok = take_item(i, wk, p, ctl, static_cast<int>(threadIdx.x & 31));
+      if (!ok || wk.qblk < 0) break;
+    } else {
+      const int w = work_rank(i);
+      if (w >= p.num_work) break;
+      wk = decode_work<kRanges>(w, p);
+    }
     const TileRange r[2] = {tile_range<kRanges>(wk, 0, p), tile_range<kRanges>(wk, 1, p)};
     const bool live0 = live<kRanges>(r[0]), live1 = live<kRanges>(r[1]);
     int lo, hi;
@@ -592,9 +660,15 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
   uint32_t s_phase = 0, o_phase = 0;
 
   for (int i = 0;; ++i) {
-    const int w = work_rank(i);
-    if (w >= p.num_work) break;
-    const WorkItem wk = decode_work<kRanges>(w, p);
+    WorkItem wk;
+    if constexpr (kRanges) {
+      if (!take_item(i, wk, p, ctl, lane)) return;
+      if (wk.qblk < 0) break;
+    } else {
+      const int w = work_rank(i);
+      if (w >= p.num_work) break;
+      wk = decode_work<kRanges>(w, p);
+    }
     const TileRange r = tile_range<kRanges>(wk, t, p);
     if (!r.active) continue;
     const int qrow = r.q0 + row_in_tile;
@@ -779,11 +853,14 @@ __device__ void softmax_role(int t, const FwdParams& p, SharedCtl* ctl, uint32_t
 // row q0 + r's visible keys [max(key_lo, 0, window start), min(key_hi, N,
 // row + 1 when causal)) and the block reduces them to the span of K/V tiles
 // [lo / 128, ceil(hi / 128)) that covers every non-empty row; (0, 0) when
-// no row of the tile sees a key.
+// no row of the tile sees a key.  It also zeroes the attention kernel's
+// item counter (dynamic deal), when there is one.
 __global__ void __launch_bounds__(128) row_range_tiles_kernel(const int* __restrict__ key_lo,
                                                               const int* __restrict__ key_hi, int2* tile_kv,
-                                                              int N, int num_qtiles, int causal, int window) {
+                                                              int* item_counter, int N, int num_qtiles, int causal,
+                                                              int window) {
   __shared__ int s_lo[4], s_hi[4];
+  if (item_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;
   const int b = blockIdx.x / num_qtiles;
   const int qt = blockIdx.x - b * num_qtiles;
   const int row = qt * 128 + static_cast<int>(threadIdx.x);
@@ -890,6 +967,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       mbar_init(&ctl->o_empty[t], 4);
     }
     mbar_init(&ctl->drain, 1);
+    if constexpr (kRanges) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&ctl->item_full[s], 1);
+        mbar_init(&ctl->item_empty[s], 9);  // the MMA warp and the eight softmax warps
+      }
+    }
     ctl->abort = 0;
     fence_mbar_init();
   }

@@ -102,7 +102,7 @@ int backward_impl(const void* q, const void* k, const void* v, const void* o, co
   int2* tile_q = ranges ? tile_kv + static_cast<size_t>(B) * num_tiles : nullptr;
   if (ranges) {
     ea::row_range_tiles_kernel<<<static_cast<unsigned>(B * num_tiles), 128, 0, stream>>>(
-        key_lo, key_hi, tile_kv, N, static_cast<int>(num_tiles), causal, window > 0 ? window : 0);
+        key_lo, key_hi, tile_kv, nullptr, N, static_cast<int>(num_tiles), causal, window > 0 ? window : 0);
     const long long tt = static_cast<long long>(B) * num_tiles;
     ea::key_tile_queries_kernel<<<static_cast<unsigned>((tt + 127) / 128), 128, 0, stream>>>(
         tile_kv, tile_q, B, static_cast<int>(num_tiles));

@@ -46,6 +46,7 @@ int g_noalloc_sms[kMaxDevices] = {};
 unsigned long long g_timeout_ns = 2000000000ull;
 int g_max_ctas = 0;
 int g_order = 0;
+int g_item_deal = 0;
 int g_skip_arrive_once = 0;
 
 
@@ -250,8 +251,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int forward_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, int causal, int window, const int* key_lo, const int* key_hi, const int2* tile_kv,
-                   const int* item_order, int num_qtiles, float scale, int dtype, const float* q_scale,
-                   const float* k_scale, const float* v_scale, DeviceState* ds, cudaStream_t stream);
+                   const int* item_order, int* item_counter, int num_qtiles, float scale, int dtype,
+                   const float* q_scale, const float* k_scale, const float* v_scale, DeviceState* ds,
+                   cudaStream_t stream);
 
 // The forward behind attn_fwd (key_lo == key_hi == null) and attn_fwd_masked:
 // argument checks, the per-tile range pre-pass when row ranges are given,
@@ -304,19 +306,24 @@ int forward_impl(const void* q, const void* k, const void* v, void* o, float* ls
 
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
   // Per-row key ranges: reduce them to a K/V tile range per 128-row query
-  // tile, then rank the (batch, query block) pairs by cost (stream-ordered
-  // scratch from the pool, freed after the launch).
+  // tile (the same pre-pass zeroes the item counter of the dynamic deal),
+  // or rank the (batch, query block) pairs by cost (stream-ordered scratch
+  // from the pool, freed after the launch).
   int2* tile_kv = nullptr;
   int* order = nullptr;
+  int* counter = nullptr;
   if (ranges) {
     const long long pairs = static_cast<long long>(B) * num_qblk;
     const size_t tb = static_cast<size_t>(B) * num_qtiles * sizeof(int2);
     const size_t ob = static_cast<size_t>(pairs) * sizeof(int);
     void* scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, tb + ob, ds->pool, stream) != cudaSuccess) return EA_ENOMEM;
+    if (cudaMallocFromPoolAsync(&scratch, tb + ob + sizeof(int), ds->pool, stream) != cudaSuccess) return EA_ENOMEM;
     tile_kv = static_cast<int2*>(scratch);
+    // The dynamic deal numbers items past the CTA count; that stays in int.
+    if (g_order == 0 && g_item_deal == 0 && B * Hq * num_qblk + ds->num_sms < INT_MAX)
+      counter = reinterpret_cast<int*>(static_cast<char*>(scratch) + tb + ob);
     ea::row_range_tiles_kernel<<<static_cast<unsigned>(B * num_qtiles), 128, 0, stream>>>(
-        key_lo, key_hi, tile_kv, N, static_cast<int>(num_qtiles), causal, window > 0 ? window : 0);
+        key_lo, key_hi, tile_kv, counter, N, static_cast<int>(num_qtiles), causal, window > 0 ? window : 0);
     rc = cudaGetLastError() == cudaSuccess ? EA_OK : EA_ELAUNCH;
     if (rc == EA_OK && pairs <= ea::kOrderMaxPairs && g_order == 2) {
       int pow2 = 1;
@@ -344,7 +351,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* o, float* ls
       return rc;
     }
   }
-  rc = forward_launch(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, key_lo, key_hi, tile_kv, order,
+  rc = forward_launch(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, window, key_lo, key_hi, tile_kv, order, counter,
                       static_cast<int>(num_qtiles), scale, dtype, q_scale, k_scale, v_scale, ds, stream);
   if (tile_kv) cudaFreeAsync(tile_kv, stream);
   return rc;
@@ -352,8 +359,9 @@ int forward_impl(const void* q, const void* k, const void* v, void* o, float* ls
 
 int forward_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, int causal, int window, const int* key_lo, const int* key_hi, const int2* tile_kv,
-                   const int* item_order, int num_qtiles, float scale, int dtype, const float* q_scale,
-                   const float* k_scale, const float* v_scale, DeviceState* ds, cudaStream_t stream) {
+                   const int* item_order, int* item_counter, int num_qtiles, float scale, int dtype,
+                   const float* q_scale, const float* k_scale, const float* v_scale, DeviceState* ds,
+                   cudaStream_t stream) {
   const bool fp8 = dtype == EA_FP8_E4M3;
   const long long num_qblk = (N + 255) / 256;
   int rc = EA_OK;
@@ -362,6 +370,7 @@ int forward_launch(const void* q, const void* k, const void* v, void* o, float* 
   p.key_hi = key_hi;
   p.tile_kv = tile_kv;
   p.item_order = item_order;
+  p.item_counter = item_counter;
   p.num_qtiles = num_qtiles;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
@@ -495,6 +504,11 @@ int attn_set_option(int option, long long value) {
       if (value != 0 && value != 1) return EA_EINVAL;
       g_skip_arrive_once = static_cast<int>(value);
       return EA_OK;
+    case EA_OPT_ITEM_DEAL:
+      if (value != 0 && value != 1) return EA_EINVAL;
+      g_item_deal = static_cast<int>(value);
+      return EA_OK;
+
     default:
       return EA_EINVAL;
   }

@@ -55,6 +55,11 @@ def test_options_validation(lib):
     assert lib.attn_set_option(B.EA_OPT_SCHEDULE_ORDER, 0) == B.EA_OK
     assert lib.attn_set_option(B.EA_OPT_WAIT_TIMEOUT_NS, 2_000_000_000) == B.EA_OK
     assert lib.attn_set_option(B.EA_OPT_MAX_CTAS, 0) == B.EA_OK
+    assert lib.attn_set_option(B.EA_OPT_ITEM_DEAL, 2) == B.EA_EINVAL
+    assert lib.attn_set_option(B.EA_OPT_ITEM_DEAL, -1) == B.EA_EINVAL
+    assert lib.attn_set_option(B.EA_OPT_ITEM_DEAL, 1) == B.EA_OK
+    assert lib.attn_set_option(B.EA_OPT_ITEM_DEAL, 0) == B.EA_OK
+    assert lib.attn_set_option(6, 0) == B.EA_EINVAL
 
 
 # Fake but 16-byte-aligned addresses: every check below fails before any

@@ -147,8 +147,9 @@ def test_masked_runs_repeat_bitwise():
 
 def test_ranked_and_unranked_schedules_agree_bitwise():
     """The schedule (default, lightest first, or (batch, query block) pairs
-    ranked by cost) only changes which CTA takes which item: all three give
-    bit-identical results, on a batch of many pairs with unequal costs."""
+    ranked by cost; items taken from a counter or dealt statically; any CTA
+    count) only changes which CTA takes which item: all give bit-identical
+    results, on a batch of many pairs with unequal costs."""
     from exact_io_aware_78_b200 import _binding as Bn
     B, H, N, d = 24, 2, 1536, 64
     inp = make_inputs(B, H, H, N, d, "bf16", 95)
@@ -162,6 +163,17 @@ def test_ranked_and_unranked_schedules_agree_bitwise():
         finally:
             lib.attn_set_option(Bn.EA_OPT_SCHEDULE_ORDER, 0)
         assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    # the dynamic deal (the default with ranges) against the static one, and
+    # under CTA counts that make each CTA take many items from the counter
+    for deal, ctas in [(1, 0), (0, 1), (0, 5), (1, 5), (0, 0)]:
+        assert lib.attn_set_option(Bn.EA_OPT_ITEM_DEAL, deal) == 0
+        assert lib.attn_set_option(Bn.EA_OPT_MAX_CTAS, ctas) == 0
+        try:
+            b = _raw(inp, True, 0, lo, hi)
+        finally:
+            lib.attn_set_option(Bn.EA_OPT_ITEM_DEAL, 0)
+            lib.attn_set_option(Bn.EA_OPT_MAX_CTAS, 0)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]), (deal, ctas)
     q, k, v = oracle_view(inp, "bf16")
     rows = list(range(0, N, 97)) + [N - 1]
     Oref, Lref = attention_ref(q, k, v, True, 0, d ** -0.5, rows=rows, key_lo=lo.numpy(), key_hi=hi.numpy())
