@@ -60,6 +60,7 @@ struct BwdParams {
   float scale;
   int num_tiles;        // ceil(N / 128)
   int num_work;
+  int* item_counter;    // range variant: this launch's dynamic-deal counter (zeroed before the launch), or null
   unsigned long long timeout_ns;
 };
 
@@ -76,7 +77,9 @@ enum : int {
   kSiteBwdCompDp = 29,
   kSiteBwdCompAcc = 30,
   kSiteBwdDrain = 31,
-  kSiteBwdCompStats = 32
+  kSiteBwdCompStats = 32,
+  kSiteBwdItemFull = 33,   // range variant: a consumer waiting for the next work item
+  kSiteBwdItemEmpty = 34   // range variant: the load warp waiting for a free item slot
 };
 
 // ------------------------------------------------------------ preprocessing
@@ -129,6 +132,8 @@ struct BwdCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  uint64_t item_full[2], item_empty[2];  // range variant: work-item slots (load warp -> other roles)
+  int item[2];
 };
 static_assert(sizeof(BwdCtl) <= 1024, "control block");
 
@@ -153,6 +158,46 @@ __device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, BwdCtl*
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   return bwd_wait_slow(a, parity, ctl, p, site, honor_abort);
+}
+
+// Range variant: the load warp takes the CTA's i-th work item and publishes
+// its rank in slot i % 2 for the MMA warp and the eight compute warps (as
+// the forward's range kernel does).  With a counter the rank is the CTA's
+// own block index first, then gridDim.x plus the counter's next value (a
+// dynamic deal: per-row key ranges give items unequal costs in no order);
+// without one, the static deal's rank.  A rank >= num_work ends the walk.
+__device__ __forceinline__ bool bwd_publish_rank(int i, int& w, const BwdParams& p, BwdCtl* ctl) {
+  w = p.item_counter == nullptr ? work_rank(i)
+      : i == 0                  ? static_cast<int>(blockIdx.x)
+                                : static_cast<int>(gridDim.x) + atomicAdd(p.item_counter, 1);
+  const int s = i & 1;
+  if (!bwd_wait(&ctl->item_empty[s], ((static_cast<uint32_t>(i) >> 1) & 1u) ^ 1u, ctl, p, kSiteBwdItemEmpty))
+    return false;
+  ctl->item[s] = w;  // ordered before the arrive by its memory clobber
+  mbar_arrive(&ctl->item_full[s]);
+  return true;
+}
+
+// Every lane of a consumer warp calls this; lane 0 frees the slot once the
+// whole warp has read it.
+__device__ __forceinline__ bool bwd_take_rank(int i, int& w, const BwdParams& p, BwdCtl* ctl) {
+  const int s = i & 1;
+  if (!__all_sync(0xFFFFFFFFu, bwd_wait(&ctl->item_full[s], (static_cast<uint32_t>(i) >> 1) & 1u, ctl, p,
+                                        kSiteBwdItemFull)))
+    return false;
+  w = ctl->item[s];  // read after the wait (its asm has a memory clobber)
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->item_empty[s]);
+  return true;
+}
+
+// Both item slots' barriers (range variant): one producer arrival, nine
+// consumer arrivals (the MMA warp and the eight compute warps).
+__device__ __forceinline__ void bwd_init_item_slots(BwdCtl* ctl) {
+  for (int s = 0; s < 2; ++s) {
+    mbar_init(&ctl->item_full[s], 1);
+    mbar_init(&ctl->item_empty[s], 9);
+  }
 }
 
 __device__ __forceinline__ bool bwd_warp_wait(uint64_t* bar, uint32_t parity, BwdCtl* ctl, const BwdParams& p,
@@ -189,10 +234,15 @@ struct BwdCfg {
 // ------------------------------------------- per-key-tile query tiles (ranges)
 // With per-row key ranges, tile_q[b, kt] = the span [x, y) of query tiles
 // whose K/V tile range (tile_kv, from row_range_tiles_kernel) contains key
-// tile kt; (0, 0) when none does.  One thread per (b, kt).
+// tile kt; (0, 0) when none does.  One thread per (b, kt).  It also zeroes
+// the dK/dV and dQ kernels' item counters (dynamic deal), when given.
 __global__ void __launch_bounds__(128) key_tile_queries_kernel(const int2* __restrict__ tile_kv, int2* tile_q, int B,
-                                                               int num_tiles) {
+                                                               int num_tiles, int* item_counters) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (item_counters != nullptr && t == 0) {
+    item_counters[0] = 0;
+    item_counters[1] = 0;
+  }
   if (t >= static_cast<long long>(B) * num_tiles) return;
   const int b = static_cast<int>(t / num_tiles);
   const int kt = static_cast<int>(t - static_cast<long long>(b) * num_tiles);
@@ -254,7 +304,13 @@ __device__ void dkdv_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, 
   uint32_t kv_armed = 0, st_armed[2] = {0, 0}, step = 0, items = 0;
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      ok = bwd_publish_rank(i, w, p, ctl);
+      if (!ok) break;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const KvItem it = kv_item<kRanges>(w, p);
     if (it.steps == 0) continue;
@@ -321,7 +377,13 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
   uint32_t step = 0, items = 0, ph_p = 0, ph_ds = 0;
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      ok = bwd_take_rank(i, w, p, ctl);
+      if (!ok) break;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const KvItem it = kv_item<kRanges>(w, p);
     if (it.steps == 0) continue;
@@ -415,7 +477,12 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
   const float cs = p.scale_log2;
   uint32_t step = 0, items = 0, ph_s = 0, ph_dp = 0;
   for (int i = 0;; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      if (!bwd_take_rank(i, w, p, ctl)) return;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const KvItem it = kv_item<kRanges>(w, p);
     const int j = it.kt * 128 + r;  // this thread's key
@@ -598,6 +665,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&ctl->stats_ready[0], 8);
     mbar_init(&ctl->stats_ready[1], 8);
     mbar_init(&ctl->drain, 1);
+    if constexpr (kRanges) bwd_init_item_slots(ctl);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -673,7 +741,13 @@ __device__ void dq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, co
   uint32_t res_armed = 0, st_armed[2] = {0, 0}, step = 0, items = 0;
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      ok = bwd_publish_rank(i, w, p, ctl);
+      if (!ok) break;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const QItem it = q_item<kRanges>(w, p);
     if (kRanges && it.kt_hi <= it.kt_lo) continue;  // no key visible to this tile: dQ = 0
@@ -735,7 +809,13 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
   uint32_t step = 0, items = 0, ph_free = 0, ph_ds = 0;
   bool ok = true;
   for (int i = 0; ok; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      ok = bwd_take_rank(i, w, p, ctl);
+      if (!ok) break;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const QItem it = q_item<kRanges>(w, p);
     const int n = it.kt_hi - it.kt_lo;
@@ -801,7 +881,12 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
   const float cs = p.scale_log2;
   uint32_t items = 0, ph_s = 0, ph_dp = 0;
   for (int i = 0;; ++i) {
-    const int w = work_rank(i);
+    int w;
+    if constexpr (kRanges) {
+      if (!bwd_take_rank(i, w, p, ctl)) return;
+    } else {
+      w = work_rank(i);
+    }
     if (w >= p.num_work) break;
     const QItem it = q_item<kRanges>(w, p);
     const int qrow = it.qt * 128 + r;
@@ -935,6 +1020,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&ctl->stats_ready[0], 8);
     mbar_init(&ctl->stats_ready[1], 8);
     mbar_init(&ctl->drain, 1);
+    if constexpr (kRanges) bwd_init_item_slots(ctl);
     ctl->abort = 0;
     fence_mbar_init();
   }

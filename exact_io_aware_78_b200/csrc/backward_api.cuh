@@ -34,11 +34,13 @@ int launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   });
   if (rc != EA_OK) return rc;
   ea::BwdParams p = base;
+  p.item_counter = base.item_counter;  // counters[0]: dK/dV items, counters[1]: dQ items (dynamic deal)
   p.num_work = p.B * p.Hkv * p.num_tiles;  // (batch, kv head, key tile)
   int grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
   ea::attn_bwd_dkdv_sm100<kD, kRanges><<<grid, G::kThreads, G::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return EA_ELAUNCH;
+  p.item_counter = base.item_counter != nullptr ? base.item_counter + 1 : nullptr;
   p.num_work = p.B * p.Hq * p.num_tiles;  // (batch, query head, query tile)
   grid = p.num_work < ds.num_sms ? p.num_work : ds.num_sms;
   if (g_max_ctas > 0 && grid > g_max_ctas) grid = g_max_ctas;
@@ -89,23 +91,28 @@ int backward_impl(const void* q, const void* k, const void* v, const void* o, co
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
 
   // ---- per-row statistics (-LSE log2 e, D), and with row ranges the two
-  // tile tables, in stream-ordered pool scratch
+  // tile tables and the two kernels' item counters (dynamic deal), in
+  // stream-ordered pool scratch
   const long long rows = static_cast<long long>(B) * N * Hq;
   const size_t stats_bytes = static_cast<size_t>(rows) * sizeof(float2);
   const size_t table_bytes = static_cast<size_t>(B) * num_tiles * sizeof(int2);
   void* scratch = nullptr;
-  if (cudaMallocFromPoolAsync(&scratch, stats_bytes + (ranges ? 2 * table_bytes : 0), ds->pool, stream) !=
-      cudaSuccess)
+  if (cudaMallocFromPoolAsync(&scratch, stats_bytes + (ranges ? 2 * table_bytes + 2 * sizeof(int) : 0), ds->pool,
+                              stream) != cudaSuccess)
     return EA_ENOMEM;
   float2* stats = static_cast<float2*>(scratch);
   int2* tile_kv = ranges ? reinterpret_cast<int2*>(static_cast<char*>(scratch) + stats_bytes) : nullptr;
   int2* tile_q = ranges ? tile_kv + static_cast<size_t>(B) * num_tiles : nullptr;
+  int* counters = nullptr;
+  // The dynamic deal numbers items past the CTA count; that stays in int.
+  if (ranges && g_item_deal == 0 && static_cast<long long>(B) * Hq * num_tiles + ds->num_sms < INT_MAX)
+    counters = reinterpret_cast<int*>(tile_q + static_cast<size_t>(B) * num_tiles);
   if (ranges) {
     ea::row_range_tiles_kernel<<<static_cast<unsigned>(B * num_tiles), 128, 0, stream>>>(
         key_lo, key_hi, tile_kv, nullptr, N, static_cast<int>(num_tiles), causal, window > 0 ? window : 0);
     const long long tt = static_cast<long long>(B) * num_tiles;
     ea::key_tile_queries_kernel<<<static_cast<unsigned>((tt + 127) / 128), 128, 0, stream>>>(
-        tile_kv, tile_q, B, static_cast<int>(num_tiles));
+        tile_kv, tile_q, B, static_cast<int>(num_tiles), counters);
     if (cudaGetLastError() != cudaSuccess) {
       cudaFreeAsync(scratch, stream);
       return EA_ELAUNCH;
@@ -137,6 +144,7 @@ int backward_impl(const void* q, const void* k, const void* v, const void* o, co
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.num_tiles = static_cast<int>(num_tiles);
+    p.item_counter = counters;
     p.timeout_ns = g_timeout_ns;
     p.key_lo = key_lo;
     p.key_hi = key_hi;

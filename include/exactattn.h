@@ -222,12 +222,13 @@ const char* attn_status_string(int status);
  *   EA_OPT_SKIP_ARRIVE_ONCE test hook: the next launch's load warp skips its
  *                           first key/value copy, so the consumer's bounded
  *                           wait runs out and reports EA_EDEVICE_TIMEOUT.
- *   EA_OPT_ITEM_DEAL        0 (default) = with per-row key ranges and order 0,
- *                           each CTA takes its next work item from a global
- *                           counter when it finishes one (dynamic deal: the
- *                           costs of ranged items follow no order, so a
- *                           static deal leaves SMs idle); 1 = the static
- *                           boustrophedon deal everywhere.
+ *   EA_OPT_ITEM_DEAL        0 (default) = with per-row key ranges (forward
+ *                           with order 0, and backward), each CTA takes its
+ *                           next work item from a global counter when it
+ *                           starts one (dynamic deal: the costs of ranged
+ *                           items follow no order, so a static deal leaves
+ *                           SMs idle); 1 = the static boustrophedon deal
+ *                           everywhere.
  *   Results depend on neither the order nor the deal (each work item's
  *   arithmetic is the same wherever it runs).
  * Returns EA_OK or EA_EINVAL.

@@ -207,3 +207,35 @@ def test_ranges_reproducing_causal_give_the_causal_backward_bitwise():
     b = ea.backward(q, k, v, o, lse, do, causal=False, key_lo=torch.zeros_like(i).to(dev), key_hi=(i + 1).to(dev))
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_range_backward_dynamic_and_static_deals_agree_bitwise():
+    """With row ranges both backward kernels take their work items from a
+    counter (dynamic deal) by default: the gradients are bit-identical to the
+    static deal's and to any CTA count's, on documents of unequal lengths
+    (one key tile's or query tile's work is the same wherever it runs)."""
+    from exact_io_aware_78_b200 import _binding as Bn
+    B, Hq, Hkv, N, d = 3, 4, 2, 1500, 128
+    inp = inputs(B, Hq, Hkv, N, d, 7400)
+    lo, hi = make_row_ranges("documents", B, N, 7401, 30, 700)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    klo, khi = lo.to(dev), hi.to(dev)
+    o, lse = ea.forward(q, k, v, causal=True, key_lo=klo, key_hi=khi)
+    ref = ea.backward(q, k, v, o, lse, do, causal=True, key_lo=klo, key_hi=khi)
+    lib = ea.load_library()
+    try:
+        for deal, ctas in [(1, 0), (0, 1), (0, 6), (1, 6), (0, 0)]:
+            assert lib.attn_set_option(Bn.EA_OPT_ITEM_DEAL, deal) == 0
+            assert lib.attn_set_option(Bn.EA_OPT_MAX_CTAS, ctas) == 0
+            got = ea.backward(q, k, v, o, lse, do, causal=True, key_lo=klo, key_hi=khi)
+            for x, y in zip(ref, got):
+                assert torch.equal(x, y), (deal, ctas)
+    finally:
+        lib.attn_set_option(Bn.EA_OPT_ITEM_DEAL, 0)
+        lib.attn_set_option(Bn.EA_OPT_MAX_CTAS, 0)
+    scale = d ** -0.5
+    q64, k64, v64, do64 = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    O, L = attention_ref(q64, k64, v64, True, 0, scale, key_lo=lo.numpy(), key_hi=hi.numpy())
+    bref = attention_bwd_ref(q64, k64, v64, do64, True, 0, scale, key_lo=lo.numpy(), key_hi=hi.numpy(), o=O, lse=L)
+    compare(ref, bref, "documents, dynamic deal")
