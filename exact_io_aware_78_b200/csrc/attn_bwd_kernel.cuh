@@ -364,14 +364,15 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
   constexpr int kHalf = 4;  // 8 MMAs of 16 rows make one 128-row K extent
   const uint32_t k_lo = sw128_desc_lo(smem_u32(smem + G::kResOffset), 16);
   const uint32_t v_lo = sw128_desc_lo(smem_u32(smem + G::kResOffset + G::kTileBytes), 16);
-  uint32_t st_lo[2], st_mn[2], do_lo[2], do_mn[2];
-  for (int t = 0; t < 2; ++t) {
-    const uint32_t base = smem_u32(smem + G::kStageOffset + t * 2 * G::kTileBytes);
-    st_lo[t] = sw128_desc_lo(base, 16);                              // Q(s), K-major
-    st_mn[t] = sw128_desc_lo(base, C::kChunkBytes);                  // Q(s), MN-major
-    do_lo[t] = sw128_desc_lo(base + G::kTileBytes, 16);              // dO(s), K-major
-    do_mn[t] = sw128_desc_lo(base + G::kTileBytes, C::kChunkBytes);  // dO(s), MN-major
-  }
+  // Descriptors of stage 0; stage 1 sits 2 tiles further, i.e. its start
+  // address field (address >> 4, 14 bits, no carry below 256 KB) is larger
+  // by kStageStep.  Computed, not indexed, so they stay in registers.
+  const uint32_t base0 = smem_u32(smem + G::kStageOffset);
+  const uint32_t st_lo0 = sw128_desc_lo(base0, 16);                              // Q(s), K-major
+  const uint32_t st_mn0 = sw128_desc_lo(base0, C::kChunkBytes);                  // Q(s), MN-major
+  const uint32_t do_lo0 = sw128_desc_lo(base0 + G::kTileBytes, 16);              // dO(s), K-major
+  const uint32_t do_mn0 = sw128_desc_lo(base0 + G::kTileBytes, C::kChunkBytes);  // dO(s), MN-major
+  constexpr uint32_t kStageStep = (2 * G::kTileBytes) >> 4;
   const uint32_t tS = tmem + G::kColS, tDp = tmem + G::kColDp;
   const uint32_t tDv = tmem + G::kColA0, tDk = tmem + G::kColA1;
   uint32_t step = 0, items = 0, ph_p = 0, ph_ds = 0;
@@ -392,9 +393,9 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
     // prologue: S^T(0), dP^T(0)
     ok = bwd_warp_wait(&ctl->st_full[step & 1], (step >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
     if (!ok) break;
-    mma_qk<C, 0>(tS, k_lo, st_lo[step & 1], kIdS);
+    mma_qk<C, 0>(tS, k_lo, st_lo0 + (step & 1) * kStageStep, kIdS);
     mma_commit_elect(&ctl->s_full);
-    mma_qk<C, 0>(tDp, v_lo, do_lo[step & 1], kIdS);
+    mma_qk<C, 0>(tDp, v_lo, do_lo0 + (step & 1) * kStageStep, kIdS);
     mma_commit_elect(&ctl->dp_full);
     for (int s = 0; s < it.steps; ++s, ++step) {
       const int t = step & 1;
@@ -407,24 +408,24 @@ __device__ void dkdv_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_
       }
       tc_fence_after();
       // A = P^T: query columns 0-63 from words [0, 32), 64-127 from [64, 96)
-      mma_pv<C, 0, kHalf>(tDv, tS, do_mn[t], kIdAcc, s > 0 ? 1u : 0u);
-      mma_pv<C, kHalf, 2 * kHalf>(tDv, tS + 32, do_mn[t], kIdAcc, 1u);
+      mma_pv<C, 0, kHalf>(tDv, tS, do_mn0 + t * kStageStep, kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, kHalf, 2 * kHalf>(tDv, tS + 32, do_mn0 + t * kStageStep, kIdAcc, 1u);
       const bool more = s + 1 < it.steps;
       if (more) {
         ok = bwd_warp_wait(&ctl->st_full[t ^ 1], ((step + 1) >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
         if (!ok) break;
-        mma_qk<C, 0>(tS, k_lo, st_lo[t ^ 1], kIdS);
+        mma_qk<C, 0>(tS, k_lo, st_lo0 + (t ^ 1) * kStageStep, kIdS);
         mma_commit_elect(&ctl->s_full);
       }
       ok = bwd_warp_wait(&ctl->ds_full, ph_ds, ctl, p, kSiteBwdMmaDs);
       if (!ok) break;
       ph_ds ^= 1u;
       tc_fence_after();
-      mma_pv<C, 0, kHalf>(tDk, tDp, st_mn[t], kIdAcc, s > 0 ? 1u : 0u);
-      mma_pv<C, kHalf, 2 * kHalf>(tDk, tDp + 32, st_mn[t], kIdAcc, 1u);
+      mma_pv<C, 0, kHalf>(tDk, tDp, st_mn0 + t * kStageStep, kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, kHalf, 2 * kHalf>(tDk, tDp + 32, st_mn0 + t * kStageStep, kIdAcc, 1u);
       mma_commit_elect(&ctl->st_empty[t]);
       if (more) {
-        mma_qk<C, 0>(tDp, v_lo, do_lo[t ^ 1], kIdS);
+        mma_qk<C, 0>(tDp, v_lo, do_lo0 + (t ^ 1) * kStageStep, kIdS);
         mma_commit_elect(&ctl->dp_full);
       }
     }
@@ -549,32 +550,60 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
         tmem_wait_ld();
       }
       // P^T: p = 2^(s cs - lse2), masked to 0; 32 packed bf16 words.
-      {
-        const uint64_t cs2 = f2_pack(cs, cs);
-        uint32_t pk[32];
+      const float4* sg4 = reinterpret_cast<const float4*>(sg);  // rows c, c + 1: (-lse2, D) each
+      const uint64_t cs2 = f2_pack(cs, cs);
+      uint32_t pk[32];
+      if constexpr (kRanges) {
+        // Row ranges mask every step: each column's test rides along with
+        // its exponentials.
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) {
           const int c = 2 * ii;
-          const float2 a = sg[c], b = sg[c + 1];
-          const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, f2_pack(a.x, b.x));
+          const float4 ab = sg4[ii];
           float y0, y1;
-          f2_unpack(y, y0, y1);
+          f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), cs2, f2_pack(ab.x, ab.z)), y0, y1);
           float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-          if (need_mask) {
-            if (c < vlo || c >= vhi) e0 = 0.0f;
-            if (c + 1 < vlo || c + 1 >= vhi) e1 = 0.0f;
-            if constexpr (kRanges) {
-              const int2 r0 = rgg[c], r1 = rgg[c + 1];
-              if (j < r0.x || j >= r0.y) e0 = 0.0f;
-              if (j < r1.x || j >= r1.y) e1 = 0.0f;
-            }
-          }
+          const int2 r0 = rgg[c], r1 = rgg[c + 1];
+          if (c < vlo || c >= vhi || j < r0.x || j >= r0.y) e0 = 0.0f;
+          if (c + 1 < vlo || c + 1 >= vhi || j < r1.x || j >= r1.y) e1 = 0.0f;
           x[c] = e0;
           x[c + 1] = e1;
           pk[ii] = pack_bf16x2(e0, e1);
         }
-        tmem_st32(tS, pk);
+      } else {
+        // Causal / window masks touch only tiles on the diagonal or the
+        // window edge: masked scores become -inf first (exponential 0), so
+        // the exponential loop has no branch and runs in batches of 8
+        // column pairs -- loads, products, exponentials, packs -- whose
+        // latencies overlap.
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < vlo || c >= vhi) x[c] = -CUDART_INF_F;
+        }
+#pragma unroll
+        for (int b8 = 0; b8 < 4; ++b8) {
+          float4 ab[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ab[i] = sg4[8 * b8 + i];
+          float e[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = 16 * b8 + 2 * i;
+            f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), cs2, f2_pack(ab[i].x, ab[i].z)), e[2 * i], e[2 * i + 1]);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) e[i] = ex2_approx(e[i]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = 16 * b8 + 2 * i;
+            x[c] = e[2 * i];
+            x[c + 1] = e[2 * i + 1];
+            pk[8 * b8 + i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+          }
+        }
       }
+      tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -595,8 +624,9 @@ __device__ void dkdv_compute(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uin
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
           const int c = 32 * k + 2 * ii;
-          const float d0 = x[c] * (__uint_as_float(dp[2 * ii]) - sg[c].y);
-          const float d1 = x[c + 1] * (__uint_as_float(dp[2 * ii + 1]) - sg[c + 1].y);
+          const float4 ab = sg4[16 * k + ii];
+          const float d0 = x[c] * (__uint_as_float(dp[2 * ii]) - ab.y);
+          const float d1 = x[c + 1] * (__uint_as_float(dp[2 * ii + 1]) - ab.w);
           pk[ii] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tDp + 16 * k, pk);
@@ -798,13 +828,13 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
   constexpr uint32_t kIdAcc = make_idesc(1, 128, kD, false, true);
   const uint32_t q_lo = sw128_desc_lo(smem_u32(smem + G::kResOffset), 16);
   const uint32_t do_lo = sw128_desc_lo(smem_u32(smem + G::kResOffset + G::kTileBytes), 16);
-  uint32_t k_lo[2], k_mn[2], v_lo[2];
-  for (int t = 0; t < 2; ++t) {
-    const uint32_t base = smem_u32(smem + G::kStageOffset + t * 2 * G::kTileBytes);
-    k_lo[t] = sw128_desc_lo(base, 16);
-    k_mn[t] = sw128_desc_lo(base, C::kChunkBytes);
-    v_lo[t] = sw128_desc_lo(base + G::kTileBytes, 16);
-  }
+  // Stage-0 descriptors; stage 1's start address field is kStageStep larger
+  // (computed, not indexed, so they stay in registers).
+  const uint32_t base0 = smem_u32(smem + G::kStageOffset);
+  const uint32_t k_lo0 = sw128_desc_lo(base0, 16);
+  const uint32_t k_mn0 = sw128_desc_lo(base0, C::kChunkBytes);
+  const uint32_t v_lo0 = sw128_desc_lo(base0 + G::kTileBytes, 16);
+  constexpr uint32_t kStageStep = (2 * G::kTileBytes) >> 4;
   const uint32_t tS = tmem + G::kColS, tDp = tmem + G::kColDp, tDq = tmem + G::kColA0;
   uint32_t step = 0, items = 0, ph_free = 0, ph_ds = 0;
   bool ok = true;
@@ -824,9 +854,9 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
     if (!ok) break;
     ok = bwd_warp_wait(&ctl->st_full[step & 1], (step >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
     if (!ok) break;
-    mma_qk<C, 0>(tS, q_lo, k_lo[step & 1], kIdS);
+    mma_qk<C, 0>(tS, q_lo, k_lo0 + (step & 1) * kStageStep, kIdS);
     mma_commit_elect(&ctl->s_full);
-    mma_qk<C, 0>(tDp, do_lo, v_lo[step & 1], kIdS);
+    mma_qk<C, 0>(tDp, do_lo, v_lo0 + (step & 1) * kStageStep, kIdS);
     mma_commit_elect(&ctl->dp_full);
     for (int s = 0; s < n; ++s, ++step) {
       const int t = step & 1;
@@ -838,7 +868,7 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
         ok = bwd_warp_wait(&ctl->st_full[t ^ 1], ((step + 1) >> 1) & 1u, ctl, p, kSiteBwdMmaStage);
         if (!ok) break;
         tc_fence_after();
-        mma_qk<C, 0>(tS, q_lo, k_lo[t ^ 1], kIdS);
+        mma_qk<C, 0>(tS, q_lo, k_lo0 + (t ^ 1) * kStageStep, kIdS);
         mma_commit_elect(&ctl->s_full);
       }
       ok = bwd_warp_wait(&ctl->ds_full, ph_ds, ctl, p, kSiteBwdMmaDs);
@@ -850,11 +880,11 @@ __device__ void dq_mma(const BwdParams& p, BwdCtl* ctl, uint8_t* smem, uint32_t 
       }
       tc_fence_after();
       // A = dS: key columns 0-63 from words [128, 160), 64-127 from [192, 224)
-      mma_pv<C, 0, 4>(tDq, tDp, k_mn[t], kIdAcc, s > 0 ? 1u : 0u);
-      mma_pv<C, 4, 8>(tDq, tDp + 32, k_mn[t], kIdAcc, 1u);
+      mma_pv<C, 0, 4>(tDq, tDp, k_mn0 + t * kStageStep, kIdAcc, s > 0 ? 1u : 0u);
+      mma_pv<C, 4, 8>(tDq, tDp + 32, k_mn0 + t * kStageStep, kIdAcc, 1u);
       mma_commit_elect(&ctl->st_empty[t]);
       if (more) {
-        mma_qk<C, 0>(tDp, do_lo, v_lo[t ^ 1], kIdS);
+        mma_qk<C, 0>(tDp, do_lo, v_lo0 + (t ^ 1) * kStageStep, kIdS);
         mma_commit_elect(&ctl->dp_full);
       }
     }
@@ -924,21 +954,22 @@ __device__ void dq_compute(const BwdParams& p, BwdCtl* ctl, uint32_t tmem, int w
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_free);
       {
+        // masked scores to -inf first (exponential 0): the loop below has
+        // no branch, so the exponentials of consecutive columns overlap
+        if (need_mask) {
+          const int vlo = key_lo - kbase, vhi = key_hi - kbase;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < vlo || c >= vhi) x[c] = -CUDART_INF_F;
+        }
         const uint64_t cs2 = f2_pack(cs, cs);
         const uint64_t nl2 = f2_pack(st.x, st.x);
-        const int vlo = key_lo - kbase, vhi = key_hi - kbase;
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, nl2);
           float y0, y1;
-          f2_unpack(y, y0, y1);
-          float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-          if (need_mask) {
-            if (c < vlo || c >= vhi) e0 = 0.0f;
-            if (c + 1 < vlo || c + 1 >= vhi) e1 = 0.0f;
-          }
-          x[c] = e0;
-          x[c + 1] = e1;
+          f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), cs2, nl2), y0, y1);
+          x[c] = ex2_approx(y0);
+          x[c + 1] = ex2_approx(y1);
         }
       }
       ok = __all_sync(0xFFFFFFFFu, bwd_wait(&ctl->dp_full, ph_dp, ctl, p, kSiteBwdCompDp));
