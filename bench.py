@@ -16,6 +16,10 @@ Other workloads: decode_* time one attn_fwd_decode call per step (key-range
 and combine kernels); bf16_doccausal_* one attn_fwd_masked call (tile-range
 pre-pass and the range variant of the forward kernel); bwd_* one attn_bwd
 call (stats pass, dK/dV kernel, dQ kernel) after an untimed forward.
+The line's e2e figure feeds the same call from pinned host memory and reads
+the results back, every step's copies inside the timed region: pipelined
+over three streams (copies in, compute, copies out; two device buffer sets)
+for the forward workloads, one stream for decode and backward.
 
 Multi-GPU: one process per GPU.  Under torchrun WORLD_SIZE must equal
 --gpus; without torchrun, --gpus N > 1 relaunches the command as a torchrun
