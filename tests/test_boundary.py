@@ -30,6 +30,27 @@ def test_header_declares_the_boundary():
          "attn_version", "attn_fwd_fp32_noalloc", "attn_fwd_decode", "attn_fwd_masked", "attn_bwd", "attn_bwd_masked"])
 
 
+def declared_constants():
+    """Every EA_* enumerator of the header with its value."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for body in re.findall(r"enum\s*\{(.*?)\}", text, flags=re.S):
+        for name, value in re.findall(r"(EA_\w+)\s*=\s*(-?\d+)", body):
+            out[name] = int(value)
+    return out
+
+
+def test_binding_constants_match_the_header():
+    """Element types, status codes and options: the Python binding carries
+    exactly the header's values, so the two cannot drift apart."""
+    consts = declared_constants()
+    assert len(consts) >= 16, consts  # 3 element types, 8 status codes, 5 options
+    for name, value in consts.items():
+        assert getattr(B, name) == value, (name, getattr(B, name, None), value)
+    m = re.search(r"#define\s+EA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u \* (\d+)u \* (\d+)u\)", open(HEADER).read())
+    assert m and int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == 16 * 1024 * 1024
+
+
 def test_library_exports_every_declared_symbol(lib_path):
     raw = ctypes.CDLL(lib_path)
     for name in declared_functions():
