@@ -127,7 +127,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * visible keys: each 128-row query tile visits only the K/V tiles spanned by
  * its rows' ranges (a small kernel reduces the ranges per tile first, into
  * stream-ordered scratch from the library's pool that goes back to the pool
- * after the launch).
+ * after the launch; the same scratch holds the counter from which the CTAs
+ * take their work items, see EA_OPT_ITEM_DEAL).
  *
  * Errors: those of attn_fwd, plus EA_EINVAL for a NULL key_lo / key_hi or
  * arrays that are not device allocations of B*N int32, EA_EALIGN for
@@ -187,7 +188,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
  * ranges as the forward.  Rows that see no key contribute nothing; keys no
  * row sees get dK = dV = 0.  The per-tile ranges (the forward's tile table
  * and, for the dK/dV kernel, the span of query tiles that see each key
- * tile) are computed by two small kernels into pool scratch.
+ * tile) are computed by two small kernels into pool scratch, which also
+ * holds the two kernels' work-item counters (see EA_OPT_ITEM_DEAL).
  * Arguments and errors: those of attn_bwd, plus EA_EINVAL for a NULL range
  * array or one that is not a device allocation of B*N int32, EA_EALIGN for
  * one that is not 4-byte aligned.
